@@ -1,0 +1,248 @@
+"""CPU oracle of the routed-expert MoE layer (test infrastructure only).
+
+Thin ctypes wrapper around ``strata_oracle.c`` (plain C, IEEE double, single
+thread). Only the tests, the smoke check and the benchmark's CPU-baseline leg
+may import this package; the library never does.
+
+Parity status of each function and the pins that fix it are listed in the
+header of ``strata_oracle.c`` and in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "strata_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math", "-std=c99"]
+
+
+def build(src: str = _SRC, out: str = _LIB, extra: tuple = ()) -> str:
+    """Compile the oracle into a shared object (gcc, no FMA contraction)."""
+    cmd = ["gcc", *CFLAGS, *extra, "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle shared object."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        if not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+            build()
+        _lib = _bind(ctypes.CDLL(_LIB))
+    return _lib
+
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+
+
+def _bind(lib):
+    lib.oracle_bf16_to_double.restype = ctypes.c_double
+    lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.oracle_fp16_to_double.restype = ctypes.c_double
+    lib.oracle_fp16_to_double.argtypes = [ctypes.c_uint16]
+    lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+    lib.oracle_dequant.argtypes = [I, I, P, P, P]
+    lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, P, P]
+    lib.oracle_router_logits.argtypes = [I, I, I, P, P, P, P]
+    lib.oracle_topk_softmax.argtypes = [I, I, I, P, P, P]
+    lib.oracle_expert_lists.argtypes = [I, I, I, P, P, P, P]
+    lib.oracle_expert_ffn.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
+    lib.oracle_moe_layer.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
+    lib.oracle_rmsnorm_bf16.argtypes = [I, P, ctypes.c_double, P]
+    lib.oracle_residual_add_f32.argtypes = [I, P, P]
+    for fn in ("oracle_dequant", "oracle_unpack_q2_tiled", "oracle_router_logits",
+               "oracle_topk_softmax", "oracle_expert_lists", "oracle_expert_ffn",
+               "oracle_moe_layer", "oracle_rmsnorm_bf16", "oracle_residual_add_f32"):
+        getattr(lib, fn).restype = None
+    return lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+# ----------------------------------------------------------------------------
+# numpy-level API
+
+
+def bf16_to_double(bits):
+    lib = load()
+    return np.array([lib.oracle_bf16_to_double(int(b)) for b in np.ravel(bits)]).reshape(np.shape(bits))
+
+
+def fp16_to_double(bits):
+    lib = load()
+    return np.array([lib.oracle_fp16_to_double(int(b)) for b in np.ravel(bits)]).reshape(np.shape(bits))
+
+
+def double_to_bf16(v):
+    lib = load()
+    return np.array([lib.oracle_double_to_bf16(float(x)) for x in np.ravel(v)], dtype=np.uint16).reshape(np.shape(v))
+
+
+def dequant(codes, scales_fp16):
+    codes = _c(codes, np.uint8)
+    sc = _c(np.asarray(scales_fp16).view(np.uint16) if np.asarray(scales_fp16).dtype == np.float16 else scales_fp16, np.uint16)
+    rows, K = codes.shape
+    W = np.empty((rows, K), dtype=np.float64)
+    load().oracle_dequant(rows, K, _p(codes), _p(sc), _p(W))
+    return W
+
+
+def unpack_q2_tiled(blob, rows: int, K: int):
+    blob = _c(blob, np.uint8)
+    assert blob.size == rows * K // 64 * 20, "blob size does not match rows x K"
+    codes = np.empty((rows, K), dtype=np.uint8)
+    scales = np.empty((rows, K // 32), dtype=np.uint16)
+    load().oracle_unpack_q2_tiled(rows, K, _p(blob), _p(codes), _p(scales))
+    return codes, scales.view(np.float16)
+
+
+def router_logits(x_bf16, W, bias=None):
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    T, d = x.shape
+    E = W.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((T, E), dtype=np.float64)
+    load().oracle_router_logits(T, d, E, _p(x), _p(W), _p(b), _p(out))
+    return out
+
+
+def topk_softmax(logits, k: int):
+    l = _c(logits, np.float64)
+    T, E = l.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    load().oracle_topk_softmax(T, E, k, _p(l), _p(idx), _p(w))
+    return idx, w
+
+
+def expert_lists(idx, E: int):
+    idx = _c(idx, np.int32)
+    T, k = idx.shape
+    off = np.empty(E + 1, dtype=np.int32)
+    tl = np.empty(T * k, dtype=np.int32)
+    sl = np.empty(T * k, dtype=np.int32)
+    load().oracle_expert_lists(T, E, k, _p(idx), _p(off), _p(tl), _p(sl))
+    return off, tl, sl
+
+
+def _sc(a):
+    a = np.asarray(a)
+    return _c(a.view(np.uint16) if a.dtype == np.float16 else a, np.uint16)
+
+
+def expert_ffn(X, ex: dict):
+    """SwiGLU expert on rows of X (double [n, d]); ex holds codes/scales."""
+    X = _c(X, np.float64)
+    n, d = X.shape
+    f = ex["gate_codes"].shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    keep = [_c(ex["gate_codes"], np.uint8), _sc(ex["gate_scales"]),
+            _c(ex["up_codes"], np.uint8), _sc(ex["up_scales"]),
+            _c(ex["down_codes"], np.uint8), _sc(ex["down_scales"])]
+    load().oracle_expert_ffn(d, f, n, _p(X), *[_p(a) for a in keep], _p(out))
+    return out
+
+
+def moe_layer(x_bf16, W, bias, experts: list, k: int):
+    """Whole layer (small shapes): returns y (double [T, d]), idx, w."""
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    T, d = x.shape
+    E = W.shape[0]
+    f = experts[0]["gate_codes"].shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    keep = []
+
+    def arr(name, conv):
+        ptrs = (ctypes.c_void_p * E)()
+        for e in range(E):
+            a = conv(experts[e][name])
+            keep.append(a)
+            ptrs[e] = a.ctypes.data
+        keep.append(ptrs)
+        return ptrs
+
+    u8 = lambda a: _c(a, np.uint8)
+    pa = [arr("gate_codes", u8), arr("gate_scales", _sc), arr("up_codes", u8),
+          arr("up_scales", _sc), arr("down_codes", u8), arr("down_scales", _sc)]
+    y = np.empty((T, d), dtype=np.float64)
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    load().oracle_moe_layer(T, d, f, E, k, _p(x), _p(W), _p(b),
+                            *[ctypes.cast(p, ctypes.c_void_p) for p in pa], _p(y), _p(idx), _p(w))
+    return y, idx, w
+
+
+def rmsnorm_bf16(x, eps: float):
+    """bf16 bits of RMSNorm(x) for each row of x (double)."""
+    x = np.atleast_2d(_c(x, np.float64))
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib = load()
+    for t in range(x.shape[0]):
+        lib.oracle_rmsnorm_bf16(x.shape[1], _p(x[t]), float(eps), _p(out[t]))
+    return out
+
+
+def residual_add_f32(x_f32, y):
+    x = _c(x_f32, np.float32).copy()
+    y = _c(y, np.float64)
+    load().oracle_residual_add_f32(x.size, _p(x), _p(y))
+    return x
+
+
+# ----------------------------------------------------------------------------
+# workload-level helpers (experts generated on demand from the seeded source)
+
+
+def route_layer(x_bf16, W, bias, k: int):
+    """Routing of every token: logits (double), idx, w, per-expert lists."""
+    logits = router_logits(x_bf16, W, bias)
+    idx, w = topk_softmax(logits, k)
+    off, tl, sl = expert_lists(idx, W.shape[0])
+    return dict(logits=logits, idx=idx, w=w, offsets=off, token_list=tl, pair_slot=sl)
+
+
+def layer_outputs(x_bf16, route: dict, tokens, expert_source):
+    """y rows for the given tokens: sum_j w[t][j] * expert_{idx[t][j]}(x_t).
+
+    ``expert_source(e)`` returns the codes/scales dict of expert e. Experts are
+    visited once each, for all requested tokens that selected them."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    d = x_bf16.shape[1]
+    idx, w = route["idx"], route["w"]
+    y = np.zeros((tokens.size, d), dtype=np.float64)
+    X = np.stack([_bf16_row(x_bf16[t]) for t in tokens]) if tokens.size else np.zeros((0, d))
+    need = {}
+    for r, t in enumerate(tokens):
+        for j in range(idx.shape[1]):
+            need.setdefault(int(idx[t, j]), []).append((r, j))
+    for e in sorted(need):
+        rows = need[e]
+        out = expert_ffn(X[[r for r, _ in rows]], expert_source(e))
+        for (r, j), o in zip(rows, out):
+            y[r] += w[tokens[r], j] * o
+    return y
+
+
+def _bf16_row(bits):
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -1,0 +1,55 @@
+"""Plausible mistakes planted in a copy of the CPU oracle must each fail at
+least one pin. This shows the pins constrain every step of the oracle (a
+dropped term, a wrong sign or index, a transposed operand, a wrong tie rule).
+The mutants are compiled from a temporary copy; the oracle itself is never
+modified. Runs without a GPU."""
+import os
+
+import pytest
+
+import oracle
+import pins_lib
+
+MUTANTS = [
+    ("code_offset", "W[(size_t)r * K + k] = (c - 1.5) * s;", "W[(size_t)r * K + k] = (c - 1.0) * s;"),
+    ("scale_block", "scales[(size_t)r * nb + k / 32]", "scales[(size_t)r * nb + k / 64]"),
+    ("silu_sign", "g / (1.0 + exp(-g))", "g / (1.0 + exp(g))"),
+    ("gate_up_swapped", "h[r] = oracle_silu(g) * u;", "h[r] = oracle_silu(u) * g;"),
+    ("down_transposed", "o += Wd[(size_t)i * f + r] * h[r];", "o += Wd[(size_t)r * d + i] * h[r];"),
+    ("no_renormalise", "w[(size_t)t * k + j] = p[r[j].idx] / ps;", "w[(size_t)t * k + j] = p[r[j].idx];"),
+    ("tie_to_higher", "return (x->idx > y->idx) - (x->idx < y->idx);", "return (x->idx < y->idx) - (x->idx > y->idx);"),
+    ("ascending_order", "if (x->key > y->key)\n        return -1;", "if (x->key > y->key)\n        return 1;"),
+    ("bias_dropped", "acc += (double)bias[e];", "acc += 0.0;"),
+    ("softmax_no_shift", "p[e] = exp(l[e] - mx);", "p[e] = exp(l[e] - mx) + 1e-3;"),
+    ("lists_slot_major", "for (int t = 0; t < T; ++t)\n            for (int j = 0; j < k; ++j)\n                if (idx[(size_t)t * k + j] == e) {",
+     "for (int j = 0; j < k; ++j)\n            for (int t = 0; t < T; ++t)\n                if (idx[(size_t)t * k + j] == e) {"),
+    ("unpack_bit", "int bit = 16 * (c % 2) + 2 * ((c % 16) / 2);", "int bit = 2 * (c % 16);"),
+    ("unpack_scale_order", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * (1 - b);"),
+    ("rms_no_mean", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
+    ("rms_eps_outside", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss / d) + eps;"),
+    ("bf16_truncate", "double r = nearbyint(v / q) * q;", "double r = trunc(v / q) * q;"),
+    ("fp16_subnormal", "v = ldexp((double)mant, -24);", "v = ldexp((double)mant, -25);"),
+    ("residual_in_double", "x[i] = (float)((double)x[i] + y[i]);", "x[i] = (float)((double)x[i] + (float)y[i] * 1.0000001);"),
+    ("combine_weight_dropped", "y[(size_t)t * d + i] += w[(size_t)t * k + j] * o[i];", "y[(size_t)t * d + i] += o[i];"),
+]
+
+
+@pytest.mark.parametrize("name,find,repl", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_fails_a_pin(tmp_path, name, find, repl):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "strata_oracle.c")).read()
+    assert src.count(find) == 1, f"mutation site for {name} not found exactly once"
+    mut = tmp_path / f"oracle_{name}.c"
+    mut.write_text(src.replace(find, repl))
+    so = oracle.build(str(mut), str(tmp_path / f"liboracle_{name}.so"))
+    saved = oracle._lib
+    oracle._lib = oracle.load(so)
+    failed = []
+    try:
+        for check in pins_lib.ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                failed.append(check.__name__)
+    finally:
+        oracle._lib = saved
+    assert failed, f"mutant {name} passed every pin"
