@@ -1,0 +1,84 @@
+// kernels.h -- host-side launchers of the sm_100a kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace strata {
+
+// Workspace of one layer handle (all device pointers, carved from one
+// allocation). Sizes are for max_tokens tokens (T) and top_k (k).
+struct Workspace {
+    uint32_t *status;     // [1]  device status word
+    int32_t *meta;        // [16] n_active, n_tiles1, n_tiles2, n_tokens, ...
+    float *logits;        // [T * E]
+    int32_t *topk_idx;    // [T * k]
+    float *topk_w;        // [T * k]
+    int32_t *counts;      // [E]
+    int32_t *offsets;     // [E + 1]
+    int32_t *token_list;  // [T * k]
+    int32_t *pair_slot;   // [T * k]
+    float *pair_w;        // [T * k]
+    int32_t *pair_of;     // [T * k]   (t, j) -> index in the sorted pair list
+    int32_t *blk_counts;  // [nblk * E] per 256-token block (prefill lists)
+    int32_t *act;         // [E] active experts (decode path)
+    float *gu_part;       // [KS * Pd * 2 * f]   decode gate/up partial sums
+    float *o_part;        // [KSD * Pd * d]      decode down partial outputs
+    void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill)
+    void *hbuf;           // fp16 [T*k * f]       SwiGLU outputs (prefill)
+    int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
+    int4 *tiles2;         // down GEMM tiles
+    void *xn;             // bf16 [T * d]         stack: normalised input
+};
+
+// meta[] slots
+enum { META_N_ACTIVE = 0, META_N_TILES1 = 1, META_N_TILES2 = 2, META_N_TOKENS = 3 };
+
+constexpr int kRouteBlock = 256;      // tokens per block of the prefill lists
+constexpr int kDecMaxT = 16;          // largest token count of the streaming path
+constexpr int kDecKS = 4;             // decode gate/up K splits (max)
+constexpr int kDecKSD = 2;            // decode down K splits
+constexpr int kGemm1N = 128;          // gate/up GEMM: max tokens per tile
+constexpr int kGemm2N = 256;          // down GEMM: max tokens per tile
+
+struct Shape {
+    int d, f, E, k;
+};
+
+struct TmaMaps {
+    CUtensorMap m[5];  // box rows 16, 32, 64, 128, 256
+};
+
+// --- routing
+void launch_router_gemv(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
+                        cudaStream_t st);
+void launch_router_gemm(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
+                        cudaStream_t st);
+void launch_route_small(const Workspace &ws, int T, const Shape &s, cudaStream_t st);
+void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
+                        cudaStream_t st);
+void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st);
+
+// --- decode experts (T <= 16)
+// stage_ev (nullable): [2] / [3] are recorded around the gate/up kernel
+void launch_decode_experts(const Workspace &ws, const void *x, const uint8_t *blob, float *y, bool accumulate,
+                           int T, const Shape &s, int num_sms, cudaStream_t st, cudaEvent_t *stage_ev);
+
+// --- prefill experts (tensor cores)
+void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
+                         const Shape &s, int num_sms, cudaStream_t st);
+void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
+                         const Shape &s, int num_sms, cudaStream_t st);
+
+// --- misc
+void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cudaStream_t st);
+void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
+                               size_t tile_stride, cudaStream_t st);
+void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st);
+
+size_t expert_bytes(const Shape &s);
+size_t down_section_offset(const Shape &s);
+
+}  // namespace strata

@@ -1,0 +1,85 @@
+// misc.cu -- RMSNorm of the stack, the device-side packer of the 2-bit
+// format, and the bounded-wait self test.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace strata {
+
+// ------------------------------------------------------------ RMSNorm
+// Stack glue (the layer recurrence x <- x + MoE(RMSNorm(x)) with unit
+// weights): out = bf16_rne(x / sqrt(mean(x^2) + eps)), one block per token.
+// sqrtf and the division are the IEEE-rounded operations.
+__global__ void __launch_bounds__(256) k_rmsnorm_bf16(const float *__restrict__ x, __nv_bfloat16 *__restrict__ out,
+                                                       int d, float eps) {
+    __shared__ float red[8];
+    const float *xr = x + (size_t)blockIdx.x * d;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < d; i += 256) ss = fmaf(xr[i], xr[i], ss);
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < 8 ? red[threadIdx.x] : 0.f;
+        v = warp_sum(v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float inv = 1.0f / sqrtf(red[0] / (float)d + eps);
+    for (int i = threadIdx.x; i < d; i += 256) out[(size_t)blockIdx.x * d + i] = __float2bfloat16_rn(xr[i] * inv);
+}
+
+void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cudaStream_t st) {
+    if (T <= 0) return;
+    k_rmsnorm_bf16<<<T, 256, 0, st>>>(x, static_cast<__nv_bfloat16 *>(out), d, eps);
+}
+
+// ------------------------------------------------------------ packer
+// One thread per (tile, row): 64 codes -> four words (column c in word c/16
+// at bit 16*(c%2) + 2*((c%16)/2)), then the row's two block scales.
+__global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales, int rows, int K,
+                              uint8_t *__restrict__ dst, size_t tile_stride) {
+    const int slices = K / 64;
+    const long long n = (long long)(rows / 128) * slices * 128;
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n) return;
+    const int i = (int)(g & 127);
+    const long long tile = g >> 7;
+    const int p = (int)(tile / slices), s = (int)(tile % slices);
+    const int r = p * 128 + i;
+    const uint8_t *cr = codes + (size_t)r * K + (size_t)s * 64;
+    uint32_t w[4] = {0, 0, 0, 0};
+#pragma unroll 4
+    for (int c = 0; c < 64; ++c) {
+        const uint32_t v = cr[c] & 3u;
+        w[c >> 4] |= v << (16 * (c & 1) + 2 * ((c & 15) >> 1));
+    }
+    uint8_t *t = dst + (size_t)tile * tile_stride;
+    *reinterpret_cast<uint4 *>(t + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+    const uint16_t *sr = scales + (size_t)r * (K / 32) + 2 * s;
+    *reinterpret_cast<uint32_t *>(t + 2048 + 4 * i) = (uint32_t)sr[0] | ((uint32_t)sr[1] << 16);
+}
+
+void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
+                               size_t tile_stride, cudaStream_t st) {
+    const long long n = (long long)(rows / 128) * (K / 64) * 128;
+    if (n <= 0) return;
+    k_pack_matrix<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(codes, scales, rows, K, dst, tile_stride);
+}
+
+// ------------------------------------------------------------ self test
+// Waits on a barrier that nothing arrives on; the bounded wait gives up
+// after timeout_ns and records the timeout in the status word.
+__global__ void k_wait_selftest(uint32_t *status, uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0, status, nullptr, timeout_ns);
+    }
+}
+
+void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(status, timeout_ns);
+}
+
+}  // namespace strata

@@ -1,0 +1,325 @@
+// prefill_gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory) for prefill chunks.
+//
+// Prompts are read in chunks of up to 8,192 tokens and the expert products
+// run on the quantised weights instead of first expanding them to FP16 in
+// memory ("Strata：把 125B 大模型塞进 12GB 显卡…", 工程细节). Here every
+// 128-row x 64-column tile of 2-bit weights is copied once per token tile
+// into shared memory (1-D bulk copy), dequantised there to fp16, and fed to
+// tcgen05.mma; the tokens of one expert (a contiguous run of the gathered,
+// expert-sorted rows) come in by 2-D tensor copies with 128-byte swizzle.
+//
+//   MODE 0 (gate/up + SwiGLU): per tile of <= 128 tokens and 128-row panel
+//     of gate and up, two accumulators G, U [128 x N] share the token
+//     operand; the epilogue writes H = silu(G) * U (fp16, pair-major).
+//   MODE 1 (down + combine): per tile of <= 256 pairs and 128-row panel of
+//     down, O = W_down H^T; the epilogue adds w * O into y[token] with fp32
+//     reductions.
+//
+// Warp roles (448 threads): warp 0 issues the copies, warp 1 issues the MMAs
+// (one thread), warps 2-5 drain the accumulators, warps 6-13 dequantise.
+// Stage ring: full (copies landed) -> aready (dequant done) -> MMA ->
+// empty (commit). Accumulators are double-buffered (accfull / accempty), so
+// the epilogue of one tile overlaps the main loop of the next.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace strata {
+
+template <int MODE>
+struct GCfg;
+template <>
+struct GCfg<0> {
+    static constexpr int NMAT = 2, NMAX = kGemm1N, STAGES = 3;
+};
+template <>
+struct GCfg<1> {
+    static constexpr int NMAT = 1, NMAX = kGemm2N, STAGES = 4;
+};
+
+constexpr int kGemmThreads = 448;
+constexpr int kDequantWarps = 8;
+
+template <int MODE>
+struct GLayout {
+    static constexpr int NMAT = GCfg<MODE>::NMAT, NMAX = GCfg<MODE>::NMAX, STAGES = GCfg<MODE>::STAGES;
+    static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // one fp16 matrix tile
+    static constexpr uint32_t B_BYTES = NMAX * 128;    // NMAX rows of 64 fp16
+    static constexpr uint32_t W_BYTES = NMAT * 2560;   // packed 2-bit tile(s)
+    static constexpr uint32_t STAGE = ((NMAT * A_BYTES + B_BYTES + W_BYTES) + 1023) / 1024 * 1024;
+    static constexpr uint32_t SMEM = STAGES * STAGE + 1024;  // + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(2 * NMAT * NMAX <= 512, "accumulators exceed tensor memory");
+};
+
+struct GemmArgs {
+    const uint8_t *blob;
+    size_t ebytes;     // bytes per expert
+    size_t sec_off;    // byte offset of this GEMM's section inside an expert
+    int K;             // reduction length (d for MODE 0, f for MODE 1)
+    int panels;        // 128-row panels of the output (f/128 or d/128)
+    int ldo;           // MODE 0: f (row length of H); MODE 1: d (row length of y)
+    const int4 *tiles;
+    const int *n_tiles;
+    __half *H;         // MODE 0 output
+    float *y;          // MODE 1 output
+    const int *token_list;
+    const float *pair_w;
+    uint32_t *status;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_constant__ TmaMaps maps, GemmArgs a) {
+    using L = GLayout<MODE>;
+    constexpr int NMAT = L::NMAT, NMAX = L::NMAX, S = L::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[S], aready[S], empty[S], accfull[2], accempty[2], fin;
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_abort;
+
+    auto A_at = [&](int st, int mat) { return smem + (size_t)st * L::STAGE + (size_t)mat * L::A_BYTES; };
+    auto B_at = [&](int st) { return smem + (size_t)st * L::STAGE + (size_t)NMAT * L::A_BYTES; };
+    auto W_at = [&](int st) { return smem + (size_t)st * L::STAGE + (size_t)NMAT * L::A_BYTES + L::B_BYTES; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = (*a.n_tiles) * a.panels;
+    const int KSTEPS = a.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&aready[i], kDequantWarps);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], 4);
+        }
+        mbar_init(&fin, 1);
+        s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < 5; ++i) prefetch_tmap(&maps.m[i]);
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int item = blockIdx.x; item < n_items && !*(volatile int *)&s_abort; item += gridDim.x) {
+                const int4 tl = a.tiles[item / a.panels];
+                const int panel = item % a.panels;
+                const int npad = (tl.z + 15) & ~15;
+                const int bsel = npad <= 16 ? 0 : npad <= 32 ? 1 : npad <= 64 ? 2 : npad <= 128 ? 3 : 4;
+                const uint32_t brows = 16u << bsel;
+                const uint8_t *wsrc = a.blob + (size_t)tl.x * a.ebytes + a.sec_off +
+                                      (size_t)panel * KSTEPS * L::W_BYTES;
+                bool ok = true;
+                for (int ks = 0; ks < KSTEPS; ++ks, ++it) {
+                    const int st = it % S;
+                    const uint32_t ph = (it / S) & 1;
+                    if (!mbar_wait(&empty[st], ph ^ 1, a.status, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[st], L::W_BYTES + brows * 128);
+                    bulk_g2s(W_at(st), wsrc + (size_t)ks * L::W_BYTES, L::W_BYTES, &full[st]);
+                    tma_load_2d(B_at(st), &maps.m[bsel], ks * 64, tl.y, &full[st]);
+                }
+                if (!ok) break;
+            }
+            // copies still in flight (only possible after an abort) land before exit
+            const uint32_t first = it > (uint32_t)S ? it - S : 0;
+            for (uint32_t j = first; j < it; ++j) mbar_wait(&full[j % S], (j / S) & 1, a.status, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, li = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
+                const int4 tl = a.tiles[item / a.panels];
+                const int npad = (tl.z + 15) & ~15;
+                const uint32_t idesc = umma_idesc_f16(128, npad);
+                const int acc = li & 1;
+                if (!mbar_wait(&accempty[acc], ((li >> 1) & 1) ^ 1, a.status, &s_abort)) break;
+                tc_fence_after();
+                const uint32_t dcol = tbase + (uint32_t)(acc * NMAT * NMAX);
+                for (int ks = 0; ks < KSTEPS; ++ks, ++it) {
+                    const int st = it % S;
+                    const uint32_t ph = (it / S) & 1;
+                    if (!mbar_wait(&aready[st], ph, a.status, &s_abort) ||
+                        !mbar_wait(&full[st], ph, a.status, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t bdesc = umma_desc_sw128(B_at(st));
+#pragma unroll
+                    for (int mat = 0; mat < NMAT; ++mat) {
+                        const uint64_t adesc = umma_desc_sw128(A_at(st, mat));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(dcol + mat * NMAX, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[st]);
+                }
+                if (ok) umma_commit(&accfull[acc]);
+            }
+            umma_commit(&fin);  // every MMA of this thread is complete before tensor memory is freed
+            mbar_wait(&fin, 0, a.status, nullptr);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int m = 32 * q + lane;
+        uint32_t li = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+            const int4 tl = a.tiles[item / a.panels];
+            const int panel = item % a.panels;
+            const int acc = li & 1;
+            if (!mbar_wait(&accfull[acc], (li >> 1) & 1, a.status, &s_abort)) break;
+            tc_fence_after();
+            const uint32_t trow = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * NMAT * NMAX);
+            const int n = tl.z, p0 = tl.y;
+            const int feat = panel * 128 + m;
+            for (int c0 = 0; c0 < n; c0 += 16) {
+                if (MODE == 0) {
+                    float g[16], u[16];
+                    tmem_ld16(trow + c0, g);
+                    tmem_ld16(trow + NMAX + c0, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < n) a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i]) * u[i]);
+                } else {
+                    float o[16];
+                    tmem_ld16(trow + c0, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < n) {
+                            const int pr = p0 + c0 + i;
+                            atomicAdd(a.y + (size_t)a.token_list[pr] * a.ldo + feat, a.pair_w[pr] * o[i]);
+                        }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+        }
+    } else {
+        // ------------------------------------------------ dequant
+        const int dt = threadIdx.x - 192;  // 0..255
+        const int row = dt & 127, sub = dt >> 7;
+        const int mat = (MODE == 0) ? sub : 0;
+        const int c_lo = (MODE == 0) ? 0 : 4 * sub, c_hi = (MODE == 0) ? 8 : 4 * sub + 4;
+        const __half2 k1027 = __floats2half2_rn(1027.f, 1027.f);
+        const __half2 khalf = __floats2half2_rn(0.5f, 0.5f);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            for (int ks = 0; ks < KSTEPS; ++ks, ++it) {
+                const int st = it % S;
+                const uint32_t ph = (it / S) & 1;
+                if (!mbar_wait(&full[st], ph, a.status, &s_abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *wt = W_at(st) + mat * 2560;
+                const uint4 cw = *reinterpret_cast<const uint4 *>(wt + 16 * row);
+                uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + 2048 + 4 * row);
+                const __half2 s01 = __hmul2(*reinterpret_cast<__half2 *>(&scb), khalf);  // (s0/2, s1/2)
+                const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint8_t *arow = A_at(st, mat) + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (c < c_lo || c >= c_hi) continue;
+                    const uint32_t w = words[c >> 1];
+                    const __half2 sc = (c < 4) ? sh0 : sh1;
+                    uint32_t out[4];
+#pragma unroll
+                    for (int pr = 0; pr < 4; ++pr) {
+                        const int mp = 4 * (c & 1) + pr;
+                        uint32_t v = (mp == 0) ? (w << 1) : (w >> (2 * mp - 1));
+                        v = (v & 0x00060006u) | 0x64006400u;  // fp16 1024 + 2c in both halves
+                        __half2 h = *reinterpret_cast<__half2 *>(&v);
+                        h = __hmul2(__hsub2(h, k1027), sc);    // (2c - 3) * s/2 = (c - 1.5) s
+                        out[pr] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aready[st]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, L::TMEM_COLS);
+    }
+}
+
+template <int MODE>
+static void launch_gemm(const TmaMaps &maps, const GemmArgs &a, int num_sms, cudaStream_t st) {
+    using L = GLayout<MODE>;
+    k_expert_gemm<MODE><<<num_sms, kGemmThreads, L::SMEM, st>>>(maps, a);
+}
+
+void init_gemm_attributes(int max_smem) {
+    static_assert(GLayout<0>::SMEM <= 232448 && GLayout<1>::SMEM <= 232448, "shared memory budget");
+    (void)max_smem;
+    cudaFuncSetAttribute(k_expert_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<0>::SMEM);
+    cudaFuncSetAttribute(k_expert_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<1>::SMEM);
+}
+
+void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
+                         const Shape &s, int num_sms, cudaStream_t st) {
+    GemmArgs a{};
+    a.blob = blob;
+    a.ebytes = expert_bytes(s);
+    a.sec_off = 0;
+    a.K = s.d;
+    a.panels = s.f / 128;
+    a.ldo = s.f;
+    a.tiles = ws.tiles1;
+    a.n_tiles = ws.meta + META_N_TILES1;
+    a.H = static_cast<__half *>(ws.hbuf);
+    a.status = ws.status;
+    (void)max_tiles;
+    launch_gemm<0>(maps, a, num_sms, st);
+}
+
+void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
+                         const Shape &s, int num_sms, cudaStream_t st) {
+    GemmArgs a{};
+    a.blob = blob;
+    a.ebytes = expert_bytes(s);
+    a.sec_off = down_section_offset(s);
+    a.K = s.f;
+    a.panels = s.d / 128;
+    a.ldo = s.d;
+    a.tiles = ws.tiles2;
+    a.n_tiles = ws.meta + META_N_TILES2;
+    a.y = y;
+    a.token_list = ws.token_list;
+    a.pair_w = ws.pair_w;
+    a.status = ws.status;
+    (void)max_tiles;
+    launch_gemm<1>(maps, a, num_sms, st);
+}
+
+}  // namespace strata

@@ -1,0 +1,404 @@
+// route.cu -- router logits, softmax top-k and per-expert token lists.
+//
+// Router ("Strata：把 125B 大模型塞进 12GB 显卡…", 代码结构: a router kernel on
+// the GPU; 10 experts per token, 核心思路). The layer's specification fixes
+// the rest: logits = W_r x (+ bias), softmax over the layer's experts, the k
+// largest with ties to the lower expert index, probabilities renormalised
+// over the k selected, and per-expert token lists for the expert kernels.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace strata {
+
+// ------------------------------------------------------------ router GEMV
+// Decode sizes (T <= 16): one warp per expert row, 16-byte coalesced loads
+// of W_r, fp32 FMA, a fixed per-row reduction order (identical rows give
+// bit-identical logits, which the tie rule relies on).
+template <int TT>
+__global__ void __launch_bounds__(128) k_router_gemv(const __nv_bfloat16 *__restrict__ x,
+                                                      const float *__restrict__ W,
+                                                      const float *__restrict__ bias, float *__restrict__ logits,
+                                                      int T, int d, int E) {
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (e >= E) return;
+    float acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+    const float4 *w4 = reinterpret_cast<const float4 *>(W + (size_t)e * d);
+    for (int i = lane; i < d / 4; i += 32) {
+        float4 w = __ldg(w4 + i);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            if (t < T) {
+                const uint2 xr = *reinterpret_cast<const uint2 *>(x + (size_t)t * d + 4 * i);
+                float x0 = __uint_as_float(xr.x << 16), x1 = __uint_as_float(xr.x & 0xffff0000u);
+                float x2 = __uint_as_float(xr.y << 16), x3 = __uint_as_float(xr.y & 0xffff0000u);
+                acc[t] = fmaf(w.x, x0, acc[t]);
+                acc[t] = fmaf(w.y, x1, acc[t]);
+                acc[t] = fmaf(w.z, x2, acc[t]);
+                acc[t] = fmaf(w.w, x3, acc[t]);
+            }
+        }
+    }
+    const float b = bias ? bias[e] : 0.f;
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+        float v = warp_sum(acc[t]);
+        if (lane == 0 && t < T) logits[(size_t)t * E + e] = v + b;
+    }
+}
+
+// ------------------------------------------------------------ router GEMM
+// Prefill sizes: tiled fp32 SIMT GEMM, logits[T x E] = X W_r^T + b.
+// 64 tokens x 64 experts per block, 16-wide K steps, 4x4 outputs per thread,
+// K summed in ascending order per output.
+__global__ void __launch_bounds__(256) k_router_gemm(const __nv_bfloat16 *__restrict__ x,
+                                                      const float *__restrict__ W,
+                                                      const float *__restrict__ bias, float *__restrict__ logits,
+                                                      int T, int d, int E) {
+    __shared__ float xs[16][64 + 4];
+    __shared__ float wsm[16][64 + 4];
+    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < d; k0 += 16) {
+        // 64 rows x 16 k of x and of W: 1024 elements each, 4 per thread
+        for (int i = threadIdx.x; i < 1024; i += 256) {
+            int r = i >> 4, kk = i & 15;
+            int t = t0 + r, e = e0 + r;
+            xs[kk][r] = (t < T) ? __bfloat162float(x[(size_t)t * d + k0 + kk]) : 0.f;
+            wsm[kk][r] = (e < E) ? W[(size_t)e * d + k0 + kk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = wsm[kk][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int t = t0 + ty * 4 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int e = e0 + tx * 4 + j;
+            if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
+        }
+    }
+}
+
+// ------------------------------------------------------------ top-k
+// One warp per token: lane l owns experts l, l+32, ... (E <= 1024). k rounds
+// of a warp arg-max over (logit descending, index ascending); only the
+// winning lane rescans its own values. Then w_j = exp(l_j - l_max) /
+// sum_{j'} exp(l_j' - l_max), which equals the softmax over all experts
+// renormalised over the selected ones.
+__device__ __forceinline__ bool rank_better(float v, int i, float bv, int bi) {
+    return v > bv || (v == bv && i < bi);
+}
+
+__device__ void warp_topk(const float *__restrict__ lrow, int E, int k, int *sel_idx, float *sel_w) {
+    const int lane = threadIdx.x & 31;
+    float v[32];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = (lane + 32 * i < E) ? lrow[lane + 32 * i] : 0.f;
+    const int nmine = (E - lane + 31) / 32;  // values this lane owns
+    auto local_best = [&](float &bv, int &bi) {
+        bv = 0.f;
+        bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i < nmine && !((taken >> i) & 1u)) {
+                int idx = lane + 32 * i;
+                if (bi == 0x7fffffff || rank_better(v[i], idx, bv, bi)) {
+                    bv = v[i];
+                    bi = idx;
+                }
+            }
+        }
+    };
+    float bv;
+    int bi;
+    local_best(bv, bi);
+    float myval = 0.f;
+    int myidx = 0;
+    float vmax = 0.f;
+    for (int j = 0; j < k; ++j) {
+        float wv = bv;
+        int wi = bi;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, wi, o);
+            bool take = (oi != 0x7fffffff) && (wi == 0x7fffffff || rank_better(ov, oi, wv, wi));
+            if (take) {
+                wv = ov;
+                wi = oi;
+            }
+        }
+        if (j == 0) vmax = wv;
+        if (lane == j) {
+            myval = wv;
+            myidx = wi;
+        }
+        if ((wi & 31) == lane) {
+            taken |= 1u << (wi >> 5);
+            local_best(bv, bi);
+        }
+    }
+    float ex = (lane < k) ? expf(myval - vmax) : 0.f;
+    float den = warp_sum(ex);
+    if (lane < k) {
+        sel_idx[lane] = myidx;
+        sel_w[lane] = ex / den;
+    }
+}
+
+// ------------------------------------------------------------ small lists
+// Decode sizes (T <= 16): one block does top-k for every token, counts,
+// exclusive scan, stable (ascending token) scatter of the (token, slot)
+// pairs and the list of active experts.
+__global__ void __launch_bounds__(512) k_route_small(Workspace ws, int T, int E, int k) {
+    __shared__ int s_idx[16 * 32];
+    __shared__ float s_w[16 * 32];
+    __shared__ int s_cnt[1024];
+    __shared__ int s_off[1025];
+    __shared__ int s_act[1024];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < T) {
+        warp_topk(ws.logits + (size_t)warp * E, E, k, s_idx + warp * 32, s_w + warp * 32);
+        __syncwarp();
+        if (lane < k) {
+            ws.topk_idx[warp * k + lane] = s_idx[warp * 32 + lane];
+            ws.topk_w[warp * k + lane] = s_w[warp * 32 + lane];
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j) c += (s_idx[t * 32 + j] == e);
+        s_cnt[e] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // E <= 1024: serial scan is a few microseconds at most
+        int run = 0, na = 0;
+        for (int e = 0; e < E; ++e) {
+            s_off[e] = run;
+            run += s_cnt[e];
+            if (s_cnt[e]) s_act[na++] = e;
+        }
+        s_off[E] = run;
+        ws.meta[META_N_ACTIVE] = na;
+        ws.meta[META_N_TOKENS] = T;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) ws.offsets[e] = s_off[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        ws.counts[e] = s_cnt[e];
+        ws.act[e] = s_act[e];  // entries past n_active are stale, never read
+    }
+    for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
+        int t = p / k, j = p % k;
+        int e = s_idx[t * 32 + j];
+        int rank = 0;
+        for (int t2 = 0; t2 < t; ++t2)
+            for (int j2 = 0; j2 < k; ++j2) rank += (s_idx[t2 * 32 + j2] == e);
+        int pos = s_off[e] + rank;
+        ws.token_list[pos] = t;
+        ws.pair_slot[pos] = j;
+        ws.pair_w[pos] = s_w[t * 32 + j];
+        ws.pair_of[p] = pos;
+    }
+}
+
+// ------------------------------------------------------------ large lists
+// Prefill sizes. (1) top-k per token, per-256-token-block expert counts.
+__global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E, int k) {
+    __shared__ int s_cnt[1024];
+    __shared__ int s_idx[8][32];
+    __shared__ float s_w[8][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += 256) s_cnt[e] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws.meta[META_N_TOKENS] = T;
+    __syncthreads();
+    const int t0 = blockIdx.x * kRouteBlock;
+    for (int i = warp; i < kRouteBlock; i += 8) {
+        int t = t0 + i;
+        if (t >= T) break;
+        warp_topk(ws.logits + (size_t)t * E, E, k, s_idx[warp], s_w[warp]);
+        __syncwarp();
+        if (lane < k) {
+            int e = s_idx[warp][lane];
+            ws.topk_idx[(size_t)t * k + lane] = e;
+            ws.topk_w[(size_t)t * k + lane] = s_w[warp][lane];
+            atomicAdd(&s_cnt[e], 1);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += 256) ws.blk_counts[(size_t)blockIdx.x * E + e] = s_cnt[e];
+}
+
+// (2) one block: expert totals, offsets, per-block bases (in place in
+// blk_counts), and the GEMM tile lists: full tiles of all experts first,
+// then the partial ones (largest work first).
+__global__ void __launch_bounds__(1024) k_lists_scan(Workspace ws, int T, int E, int max_tiles1, int max_tiles2) {
+    __shared__ int s_tot[1024];
+    __shared__ int s_off[1025];
+    __shared__ int s_f1[1025], s_p1[1025], s_f2[1025], s_p2[1025];
+    const int nblk = (T + kRouteBlock - 1) / kRouteBlock;
+    const int e = threadIdx.x;
+    int tot = 0;
+    if (e < E) {
+        for (int b = 0; b < nblk; ++b) {
+            int c = ws.blk_counts[(size_t)b * E + e];
+            ws.blk_counts[(size_t)b * E + e] = tot;  // exclusive prefix over blocks
+            tot += c;
+        }
+        s_tot[e] = tot;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0, f1 = 0, p1 = 0, f2 = 0, p2 = 0;
+        for (int i = 0; i < E; ++i) {
+            s_off[i] = run;
+            run += s_tot[i];
+            s_f1[i] = f1;
+            f1 += s_tot[i] / kGemm1N;
+            s_p1[i] = p1;
+            p1 += (s_tot[i] % kGemm1N) != 0;
+            s_f2[i] = f2;
+            f2 += s_tot[i] / kGemm2N;
+            s_p2[i] = p2;
+            p2 += (s_tot[i] % kGemm2N) != 0;
+        }
+        s_off[E] = run;
+        s_f1[E] = f1;
+        s_p1[E] = p1;
+        s_f2[E] = f2;
+        s_p2[E] = p2;
+        ws.meta[META_N_TILES1] = min(f1 + p1, max_tiles1);
+        ws.meta[META_N_TILES2] = min(f2 + p2, max_tiles2);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) ws.offsets[E] = s_off[E];
+    if (e < E) {
+        ws.offsets[e] = s_off[e];
+        ws.counts[e] = tot;
+        for (int b = 0; b < nblk; ++b) ws.blk_counts[(size_t)b * E + e] += s_off[e];
+        const int F1 = s_f1[E], F2 = s_f2[E];
+        int nf = tot / kGemm1N;
+        for (int i = 0; i < nf; ++i)
+            if (s_f1[e] + i < max_tiles1)
+                ws.tiles1[s_f1[e] + i] = make_int4(e, s_off[e] + i * kGemm1N, kGemm1N, 0);
+        if (tot % kGemm1N && F1 + s_p1[e] < max_tiles1)
+            ws.tiles1[F1 + s_p1[e]] = make_int4(e, s_off[e] + nf * kGemm1N, tot % kGemm1N, 0);
+        nf = tot / kGemm2N;
+        for (int i = 0; i < nf; ++i)
+            if (s_f2[e] + i < max_tiles2)
+                ws.tiles2[s_f2[e] + i] = make_int4(e, s_off[e] + i * kGemm2N, kGemm2N, 0);
+        if (tot % kGemm2N && F2 + s_p2[e] < max_tiles2)
+            ws.tiles2[F2 + s_p2[e]] = make_int4(e, s_off[e] + nf * kGemm2N, tot % kGemm2N, 0);
+    }
+}
+
+// (3) stable scatter: within a 256-token block, a bitmap per expert of the
+// tokens that chose it; the rank of (t, e) is the block base plus the number
+// of earlier tokens of the block in e's bitmap.
+__global__ void __launch_bounds__(256) k_lists_scatter(Workspace ws, int T, int E, int k) {
+    extern __shared__ uint32_t s_bits[];  // [E][8]
+    for (int i = threadIdx.x; i < E * 8; i += 256) s_bits[i] = 0u;
+    __syncthreads();
+    const int i = threadIdx.x;
+    const int t = blockIdx.x * kRouteBlock + i;
+    if (t < T)
+        for (int j = 0; j < k; ++j) {
+            int e = ws.topk_idx[(size_t)t * k + j];
+            atomicOr(&s_bits[e * 8 + (i >> 5)], 1u << (i & 31));
+        }
+    __syncthreads();
+    if (t < T)
+        for (int j = 0; j < k; ++j) {
+            int e = ws.topk_idx[(size_t)t * k + j];
+            int r = __popc(s_bits[e * 8 + (i >> 5)] & ((1u << (i & 31)) - 1u));
+            for (int w = 0; w < (i >> 5); ++w) r += __popc(s_bits[e * 8 + w]);
+            int pos = ws.blk_counts[(size_t)blockIdx.x * E + e] + r;
+            ws.token_list[pos] = t;
+            ws.pair_slot[pos] = j;
+            ws.pair_w[pos] = ws.topk_w[(size_t)t * k + j];
+            ws.pair_of[(size_t)t * k + j] = pos;
+        }
+}
+
+// ------------------------------------------------------------ gather
+// xp[p] = fp16(x[token_list[p]]): one warp per pair row, 16-byte accesses.
+__global__ void __launch_bounds__(256) k_gather_xp(const __nv_bfloat16 *__restrict__ x,
+                                                    const int *__restrict__ token_list, __half *__restrict__ xp,
+                                                    int npairs, int d) {
+    const int p = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (p >= npairs) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)token_list[p] * d);
+    uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)p * d);
+    for (int c = lane; c < d / 8; c += 32) {
+        uint4 v = __ldg(src + c);
+        uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float lo = __uint_as_float(in[q] << 16), hi = __uint_as_float(in[q] & 0xffff0000u);
+            __half2 h = __floats2half2_rn(lo, hi);
+            out[q] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        dst[c] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// ------------------------------------------------------------ launchers
+void launch_router_gemv(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
+                        cudaStream_t st) {
+    dim3 grid((s.E + 3) / 4), block(128);
+    auto xb = static_cast<const __nv_bfloat16 *>(x);
+    if (T <= 1)
+        k_router_gemv<1><<<grid, block, 0, st>>>(xb, W, bias, logits, T, s.d, s.E);
+    else if (T <= 4)
+        k_router_gemv<4><<<grid, block, 0, st>>>(xb, W, bias, logits, T, s.d, s.E);
+    else
+        k_router_gemv<16><<<grid, block, 0, st>>>(xb, W, bias, logits, T, s.d, s.E);
+}
+
+void launch_router_gemm(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
+                        cudaStream_t st) {
+    dim3 grid((s.E + 63) / 64, (T + 63) / 64), block(256);
+    k_router_gemm<<<grid, block, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), W, bias, logits, T, s.d, s.E);
+}
+
+void launch_route_small(const Workspace &ws, int T, const Shape &s, cudaStream_t st) {
+    k_route_small<<<1, 512, 0, st>>>(ws, T, s.E, s.k);
+}
+
+void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
+                        cudaStream_t st) {
+    const int nblk = (T + kRouteBlock - 1) / kRouteBlock;
+    k_topk_blocks<<<nblk, 256, 0, st>>>(ws, T, s.E, s.k);
+    k_lists_scan<<<1, 1024, 0, st>>>(ws, T, s.E, max_tiles1, max_tiles2);
+    k_lists_scatter<<<nblk, 256, (size_t)s.E * 8 * sizeof(uint32_t), st>>>(ws, T, s.E, s.k);
+}
+
+void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st) {
+    const int np = T * s.k;
+    k_gather_xp<<<(np + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), ws.token_list,
+                                               static_cast<__half *>(ws.xp), np, s.d);
+}
+
+}  // namespace strata

@@ -1,0 +1,240 @@
+/*
+ * strata_moe.h -- C ABI of the B200 (sm_100a) routed-expert MoE layer with
+ * 2-bit block-quantised experts.
+ *
+ * What the layer computes (sources: the pages' titles and sections):
+ *   - "Strata Skill：把 125B MoE 大模型塞进 12GB 显卡的本地推理引擎", 介绍, and
+ *     "Strata：把 125B 大模型塞进 12GB 显卡，24,576 个专家在内存与 SSD 之间流动",
+ *     核心思路: each token is served by 10 of the layer's experts.
+ *   - "Strata — 8~12GB 显存跑 125B 大模型的本地推理引擎", §5 table: 512
+ *     experts per layer; §2 and the second page's 投机解码: 48 layers, and a
+ *     decode step verifies 1 + up to 3 draft tokens in one 48-layer pass.
+ *   - the second page, 工程细节: prompts are read in chunks of up to 8,192
+ *     tokens, and the expert products run on the quantised weights without
+ *     first expanding them to FP16 in memory.
+ *   - the second page, 代码结构: a router kernel and an MoE kernel on the GPU.
+ *   The layer's specification fixes the rest: router logits l = W_r x (+ an
+ *   optional per-expert bias), softmax over the experts, the k largest
+ *   (ties to the lower expert index), their probabilities renormalised to
+ *   sum to 1; each selected expert is a SwiGLU MLP on its 2-bit weights,
+ *   h = silu(W_gate x) * (W_up x), o = W_down h; y = sum_j w_j o_j.
+ *
+ * Conventions
+ *   - All tensor arguments are DEVICE pointers unless marked "host". The
+ *     caller owns every tensor and stream; the library owns only the
+ *     workspace it allocates when strata_moe_layer_create gets NULL.
+ *   - Every compute call is asynchronous on `stream` and returns after
+ *     enqueue. Argument errors are returned synchronously and nothing is
+ *     enqueued. Device-side errors (a bounded wait that ran out) are recorded
+ *     in a device status word read by strata_moe_check_status.
+ *   - No C++ exception crosses this ABI. strata_last_error() gives a
+ *     thread-local message for the last non-OK status of the calling thread.
+ *   - Device pointers must be 16-byte aligned.
+ *   - One layer handle serves one stream at a time: its workspace holds the
+ *     routing of the last call.
+ */
+#ifndef STRATA_MOE_H
+#define STRATA_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *strata_stream_t;
+
+typedef enum {
+    STRATA_OK = 0,
+    STRATA_ERR_INVALID_ARG = -1,    /* bad pointer, size, alignment or desc */
+    STRATA_ERR_UNSUPPORTED = -2,    /* shape or flag this build does not run */
+    STRATA_ERR_CUDA = -3,           /* a CUDA runtime call failed */
+    STRATA_ERR_OOM = -4,            /* workspace allocation failed */
+    STRATA_ERR_TOO_MANY_TOKENS = -5,/* n_tokens > max_tokens (layer calls) */
+    STRATA_ERR_BAD_BLOB = -6,       /* blob pointer or packer input invalid */
+    STRATA_ERR_TIMEOUT = -7         /* a device wait exceeded its time limit */
+} strata_status;
+
+/* ------------------------------------------------------------------ format
+ * STRATA_FMT_Q2_0_TILED: the 2-bit block format ("Q2_0" on the pages, first
+ * page, 功能与原则; its bits are this library's).
+ *   weight W[r][k] = (c[r][k] - 1.5) * s[r][k/32], c in {0,1,2,3}, s fp16:
+ *   32-weight blocks along the reduction dimension K of each output row.
+ * A matrix [R x K] (R % 128 == 0, K % 64 == 0) is a sequence of tiles, one
+ * per (128-row panel p, 64-column slice s); a tile is 2560 bytes:
+ *   bytes [0, 2048):   codes, row i (0..127) at bytes 16i..16i+15, as four
+ *                      little-endian uint32 words; column c (0..63) of the
+ *                      tile lives in word c/16 at bit 16*(c%2) + 2*((c%16)/2)
+ *                      (even columns in the low halves, odd columns in the
+ *                      high halves, so one shift and mask yields two codes
+ *                      for adjacent columns);
+ *   bytes [2048, 2560): scales, row i at 2048+4i: fp16 (little-endian) of
+ *                      block 2s, then of block 2s+1.
+ * Every tile is a multiple of 16 bytes, so tiles serve 128-bit loads and
+ * 1-D bulk (TMA) copies alike; a 64-column slice of a 128-row panel, as the
+ * tensor-core path consumes it, is one contiguous tile.
+ *
+ * Expert blob: experts 0..E-1 back to back, strata_moe_expert_bytes() each:
+ *   gate/up section: for p in 0..f/128-1, for s in 0..d/64-1:
+ *                    [gate tile (p,s)][up tile (p,s)]     (5120 bytes)
+ *   down section:    down matrix [d x f] tiles in (p, s) order, p < d/128,
+ *                    s < f/64                              (2560 bytes each)
+ *   per expert: 3*d*f/32*10 bytes (d=2048, f=768: 1,474,560 bytes).
+ */
+#define STRATA_FMT_Q2_0_TILED 1
+#define STRATA_Q2_TILE_ROWS 128
+#define STRATA_Q2_TILE_COLS 64
+#define STRATA_Q2_TILE_BYTES 2560
+
+/* desc.flags */
+#define STRATA_ACCUMULATE 1u      /* y += MoE(x) instead of y = MoE(x) */
+#define STRATA_FORCE_PREFILL 2u   /* use the tensor-core path even for <= 16 tokens */
+
+/* Largest token count served by the streaming (decode/verify) path. */
+#define STRATA_DECODE_MAX_TOKENS 16
+
+typedef struct {
+    int32_t d_model;      /* d, multiple of 128 */
+    int32_t d_ff;         /* f, expert intermediate size, multiple of 128 */
+    int32_t n_experts;    /* E, 1..1024 */
+    int32_t top_k;        /* k, 1 <= k <= min(E, 32) */
+    int32_t max_tokens;   /* largest n_tokens of one layer call (workspace size) */
+    int32_t block_size;   /* must be 32 */
+    int32_t weight_format;/* must be STRATA_FMT_Q2_0_TILED */
+    uint32_t flags;       /* STRATA_ACCUMULATE | STRATA_FORCE_PREFILL */
+    const float *router_bias; /* device fp32 [E] added to the logits, or NULL */
+} strata_moe_desc;
+
+typedef struct strata_moe_layer_s *strata_moe_layer;
+
+/* Bytes of one packed matrix [rows x K] (rows % 128 == 0, K % 64 == 0). */
+size_t strata_q2_matrix_bytes(int32_t rows, int32_t K);
+/* Bytes of one packed expert: 3*d*f/32*10. */
+size_t strata_moe_expert_bytes(const strata_moe_desc *desc);
+/* Bytes of the whole expert blob of a layer: E * strata_moe_expert_bytes. */
+size_t strata_moe_expert_blob_bytes(const strata_moe_desc *desc);
+/* Device workspace a layer handle needs for desc->max_tokens tokens. */
+size_t strata_moe_workspace_bytes(const strata_moe_desc *desc);
+
+/* Validate desc and build a layer handle. workspace: device memory of at
+ * least strata_moe_workspace_bytes(desc) bytes owned by the caller, or NULL
+ * to let the library allocate (and later free) it. The current CUDA device
+ * at create time is the device every later call must run on.
+ * Errors: INVALID_ARG / UNSUPPORTED (desc), OOM, CUDA. */
+strata_status strata_moe_layer_create(const strata_moe_desc *desc, void *workspace,
+                                      size_t workspace_bytes, strata_moe_layer *out);
+/* Free the handle (and the workspace if the library allocated it). The
+ * caller must make sure no work using it is still queued. */
+strata_status strata_moe_layer_destroy(strata_moe_layer layer);
+
+/* One MoE layer: y (=|+=) sum_j w_j * SwiGLU_{e_j}(x) for every token.
+ *   x_bf16      [n_tokens x d] bf16, row-major
+ *   router_w    [E x d] fp32, row-major (router bias: desc.router_bias)
+ *   expert_blob E packed experts (format above)
+ *   y           [n_tokens x d] fp32
+ * n_tokens in 0..max_tokens (0 is a no-op). n_tokens <= 16 streams only the
+ * selected experts' weights (CUDA cores); larger calls run the grouped
+ * tensor-core GEMMs. Errors: INVALID_ARG, TOO_MANY_TOKENS, CUDA. */
+strata_status strata_moe_forward(strata_moe_layer layer, const void *x_bf16, const float *router_w,
+                                 const void *expert_blob, float *y, int32_t n_tokens,
+                                 strata_stream_t stream);
+
+/* Router logits only (step one of the layer): logits [n_tokens x E] fp32 =
+ * x W_r^T + bias. Same paths and precision as inside strata_moe_forward. */
+strata_status strata_moe_router_logits(strata_moe_layer layer, const void *x_bf16,
+                                       const float *router_w, float *logits, int32_t n_tokens,
+                                       strata_stream_t stream);
+
+/* Routing only: logits, softmax top-k, renormalised weights and the
+ * per-expert token lists, kept in the workspace for strata_moe_experts and
+ * strata_moe_get_routing. */
+strata_status strata_moe_route(strata_moe_layer layer, const void *x_bf16, const float *router_w,
+                               int32_t n_tokens, strata_stream_t stream);
+
+/* Expert computation and combine for the routing of the last
+ * strata_moe_route / strata_moe_forward call on this handle (same x and
+ * n_tokens). */
+strata_status strata_moe_experts(strata_moe_layer layer, const void *x_bf16, const void *expert_blob,
+                                 float *y, int32_t n_tokens, strata_stream_t stream);
+
+/* Copy the routing of the last call into caller buffers (device pointers;
+ * any may be NULL):
+ *   topk_idx [T x k] int32, experts of each token in rank order
+ *            (logit descending, ties to the lower index)
+ *   topk_w   [T x k] fp32, renormalised softmax weights
+ *   expert_offsets [E + 1] int32, start of each expert's list
+ *   token_list [T*k] int32, tokens of each expert in ascending order
+ *   pair_slot  [T*k] int32, slot j at which the token chose that expert */
+strata_status strata_moe_get_routing(strata_moe_layer layer, int32_t *topk_idx, float *topk_w,
+                                     int32_t *expert_offsets, int32_t *token_list,
+                                     int32_t *pair_slot, strata_stream_t stream);
+
+/* A stack of n_layers layers with the residual recurrence
+ *   x <- x + MoE_l(bf16(RMSNorm(x)))   (RMSNorm with unit weights, eps)
+ * x_resid [n_tokens x d] fp32 in/out. router_w, router_bias and
+ * expert_blobs are HOST arrays of n_layers device pointers (router_bias may
+ * be NULL, or hold NULL entries). n_tokens may exceed max_tokens: tokens are
+ * processed in chunks of max_tokens, each chunk through all layers. The
+ * decode-size sequence is captured into a CUDA graph on first use and
+ * replayed while the pointers stay the same (not when the stream is already
+ * capturing). desc.flags STRATA_ACCUMULATE is ignored here. */
+strata_status strata_moe_stack_forward(strata_moe_layer layer, int32_t n_layers,
+                                       const float *const *router_w,
+                                       const float *const *router_bias,
+                                       const void *const *expert_blobs, float *x_resid,
+                                       int32_t n_tokens, float rms_eps, strata_stream_t stream);
+
+/* RMSNorm with unit weights, rounded to bf16 (step of the stack):
+ * out[t][i] = bf16_rne(x[t][i] / sqrt(mean_i x[t][i]^2 + eps)). */
+strata_status strata_rmsnorm_bf16(const float *x, void *out_bf16, int32_t n_tokens, int32_t d,
+                                  float eps, strata_stream_t stream);
+
+/* Stage timing hook. events: HOST array of n_events cudaEvent_t handles
+ * created by the caller. With n_events == 5, every later forward / experts
+ * call on this handle records, on its stream: events[0] at its start,
+ * [1] after routing, [2] right before and [3] right after the dominant
+ * expert kernel (decode: the gate/up streaming kernel; prefill: the gate/up
+ * tensor-core GEMM), [4] at its end. n_events == 0 removes the hook.
+ * Errors: INVALID_ARG for any other count. */
+strata_status strata_moe_set_stage_events(strata_moe_layer layer, void *const *events, int32_t n_events);
+
+/* Synchronise the layer's stream work and read its device status word
+ * (OK, or TIMEOUT if a bounded device wait ran out); clears the word. */
+strata_status strata_moe_check_status(strata_moe_layer layer);
+
+/* Pack one matrix on the HOST: codes [rows x K] one code (0..3) per byte,
+ * scales [rows x K/32] fp16 bits, into dst (host, strata_q2_matrix_bytes).
+ * Errors: BAD_BLOB (a code > 3), INVALID_ARG. */
+strata_status strata_q2_pack(const uint8_t *codes, const uint16_t *scales_fp16, int32_t rows,
+                             int32_t K, void *dst);
+
+/* Pack one expert on the HOST into its blob section (dst: host,
+ * strata_moe_expert_bytes): gate/up [f x d], down [d x f]. */
+strata_status strata_moe_pack_expert(const strata_moe_desc *desc, const uint8_t *gate_codes,
+                                     const uint16_t *gate_scales, const uint8_t *up_codes,
+                                     const uint16_t *up_scales, const uint8_t *down_codes,
+                                     const uint16_t *down_scales, void *dst);
+
+/* Same as strata_moe_pack_expert with device pointers, on `stream`. Codes
+ * above 3 are masked to 2 bits. */
+strata_status strata_moe_pack_expert_device(const strata_moe_desc *desc, const uint8_t *gate_codes,
+                                            const uint16_t *gate_scales, const uint8_t *up_codes,
+                                            const uint16_t *up_scales, const uint8_t *down_codes,
+                                            const uint16_t *down_scales, void *dst,
+                                            strata_stream_t stream);
+
+/* Failure-detection self test: launches a kernel whose bounded wait polls a
+ * flag that nothing sets, for timeout_ns nanoseconds (1e3..1e10), then
+ * returns; reports STRATA_ERR_TIMEOUT through the status word like any
+ * other wait. Synchronous. */
+strata_status strata_selftest_wait_timeout(uint64_t timeout_ns, strata_stream_t stream);
+
+const char *strata_status_string(strata_status s);
+const char *strata_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STRATA_MOE_H */

@@ -55,7 +55,7 @@ def _bind(lib):
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
     lib.oracle_dequant.argtypes = [I, I, P, P, P]
-    lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, P, P]
+    lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, ctypes.c_long, P, P]
     lib.oracle_router_logits.argtypes = [I, I, I, P, P, P, P]
     lib.oracle_topk_softmax.argtypes = [I, I, I, P, P, P]
     lib.oracle_expert_lists.argtypes = [I, I, I, P, P, P, P]
@@ -106,13 +106,26 @@ def dequant(codes, scales_fp16):
     return W
 
 
-def unpack_q2_tiled(blob, rows: int, K: int):
+def unpack_q2_tiled(blob, rows: int, K: int, tile_stride: int = 2560):
+    """Codes and scales of one matrix from tiles at ``blob + t * tile_stride``."""
     blob = _c(blob, np.uint8)
-    assert blob.size == rows * K // 64 * 20, "blob size does not match rows x K"
+    ntiles = rows // 128 * (K // 64)
+    assert blob.size >= (ntiles - 1) * tile_stride + 2560, "blob too small for rows x K"
     codes = np.empty((rows, K), dtype=np.uint8)
     scales = np.empty((rows, K // 32), dtype=np.uint16)
-    load().oracle_unpack_q2_tiled(rows, K, _p(blob), _p(codes), _p(scales))
+    load().oracle_unpack_q2_tiled(rows, K, _p(blob), tile_stride, _p(codes), _p(scales))
     return codes, scales.view(np.float16)
+
+
+def unpack_expert(blob, d: int, f: int) -> dict:
+    """Codes/scales of one expert from its blob section: interleaved gate/up
+    tiles (5120-byte pairs), then the down matrix (header's layout)."""
+    blob = _c(blob, np.uint8)
+    gu = f * d // 64 * 20 * 2
+    gc, gs = unpack_q2_tiled(blob, f, d, 5120)
+    uc, us = unpack_q2_tiled(blob[2560:], f, d, 5120)
+    dc, ds = unpack_q2_tiled(blob[gu:], d, f, 2560)
+    return dict(gate_codes=gc, gate_scales=gs, up_codes=uc, up_scales=us, down_codes=dc, down_scales=ds)
 
 
 def router_logits(x_bf16, W, bias=None):

@@ -104,13 +104,16 @@ void oracle_dequant(int rows, int K, const uint8_t *codes, const uint16_t *scale
  * 2560 bytes; inside a tile, row i's 64 codes occupy bytes 16i..16i+15 as four
  * little-endian 32-bit words; column c of the tile sits in word c/16 at bit
  * 16*(c%2) + 2*((c%16)/2); the row's two fp16 scales follow at byte
- * 2048 + 4i). Returns one code per byte and the fp16 scale bits. */
-void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, uint8_t *codes, uint16_t *scales)
+ * 2048 + 4i). Tile t starts at byte t * tile_stride (2560 for a lone matrix;
+ * 5120 for the interleaved gate/up tiles of an expert). Returns one code per
+ * byte and the fp16 scale bits. */
+void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long tile_stride, uint8_t *codes,
+                            uint16_t *scales)
 {
     int slices = K / 64;
     for (int p = 0; p < rows / 128; ++p)
         for (int s = 0; s < slices; ++s) {
-            const uint8_t *tile = blob + ((size_t)p * slices + s) * 2560;
+            const uint8_t *tile = blob + ((size_t)p * slices + s) * (size_t)tile_stride;
             for (int i = 0; i < 128; ++i) {
                 int r = p * 128 + i;
                 for (int c = 0; c < 64; ++c) {

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI library (no GPU): the shared library loads,
+exports every function the header declares, its host packer writes the
+documented format (pinned by the hand-worked tile and by the oracle's
+independent unpacker), and the size / desc-validation functions behave."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import pins_lib
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "strata_moe.h")
+
+
+@pytest.fixture(scope="module")
+def S():
+    import __graft_entry__
+
+    __graft_entry__._load_builder().build()
+    import bit_quantized_moe_warp_b200 as S
+
+    return S
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(strata_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_symbols_exported(S):
+    names = header_functions()
+    assert len(names) >= 18
+    lib = ctypes.CDLL(S.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+    assert sorted(S.EXPORTED) == names, "Python binding and header disagree"
+
+
+def test_pack_golden_tile(S):
+    blob, expects = pins_lib.load_tile_example()
+    codes, scales = oracle.unpack_q2_tiled(blob, 128, 64)
+    out = np.zeros(2560, np.uint8)
+    S.strata_q2_pack(codes, scales, 128, 64, out)
+    assert np.array_equal(out, blob), "library packer differs from the hand-worked tile"
+
+
+@pytest.mark.parametrize("rows,K", [(128, 64), (256, 128), (128, 768), (384, 256)])
+def test_pack_roundtrip_matrix(S, rows, K):
+    rng = np.random.default_rng(rows * 7 + K)
+    codes = rng.integers(0, 4, (rows, K), dtype=np.uint8)
+    scales = (rng.standard_normal((rows, K // 32)) * 0.02).astype(np.float16)
+    n = S.strata_q2_matrix_bytes(rows, K)
+    assert n == rows * K // 64 * 20
+    out = np.zeros(n, np.uint8)
+    S.strata_q2_pack(codes, scales, rows, K, out)
+    c2, s2 = oracle.unpack_q2_tiled(out, rows, K)
+    assert np.array_equal(c2, codes)
+    assert np.array_equal(s2.view(np.uint16), scales.view(np.uint16))
+
+
+def test_pack_expert_layout(S):
+    d, f = 256, 128
+    desc = S.make_desc(d, f, 4, 2, 8)
+    ex = synth.gen_expert(5, 0, 3, d, f)
+    eb = S.strata_moe_expert_bytes(desc)
+    assert eb == 3 * d * f // 32 * 10
+    out = np.zeros(eb, np.uint8)
+    S.strata_moe_pack_expert(desc, ex["gate_codes"], ex["gate_scales"], ex["up_codes"], ex["up_scales"],
+                             ex["down_codes"], ex["down_scales"], out)
+    got = oracle.unpack_expert(out, d, f)
+    for key in ex:
+        a, b = got[key], ex[key]
+        if a.dtype == np.float16:
+            a, b = a.view(np.uint16), b.view(np.uint16)
+        assert np.array_equal(a, b), key
+
+
+def test_pack_rejects_bad_code(S):
+    codes = np.zeros((128, 64), np.uint8)
+    codes[3, 5] = 4
+    with pytest.raises(S.StrataError) as ei:
+        S.strata_q2_pack(codes, np.zeros((128, 2), np.float16), 128, 64, np.zeros(2560, np.uint8))
+    assert ei.value.status == S.STRATA_ERR_BAD_BLOB
+
+
+def test_desc_validation(S):
+    ok = S.make_desc(2048, 768, 512, 10, 8192)
+    assert S.strata_moe_expert_bytes(ok) == 1474560
+    assert S.strata_moe_expert_blob_bytes(ok) == 1474560 * 512
+    assert S.strata_moe_workspace_bytes(ok) > 0
+    bad = [S.make_desc(2000, 768, 512, 10, 16), S.make_desc(2048, 700, 512, 10, 16),
+           S.make_desc(2048, 768, 0, 1, 16), S.make_desc(2048, 768, 8, 9, 16),
+           S.make_desc(2048, 768, 512, 33, 16), S.make_desc(2048, 768, 512, 10, 0),
+           S.make_desc(2048, 768, 2048, 10, 16)]
+    for dsc in bad:
+        assert S.strata_moe_workspace_bytes(dsc) == 0
+        assert S.strata_moe_expert_bytes(dsc) == 0
+    d2 = S.make_desc(256, 128, 16, 4, 8)
+    d2.block_size = 16
+    assert S.strata_moe_workspace_bytes(d2) == 0
+    assert S.strata_q2_matrix_bytes(100, 64) == 0
+
+
+def test_status_strings(S):
+    for code in range(-7, 1):
+        assert S.strata_status_string(code)

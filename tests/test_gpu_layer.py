@@ -1,0 +1,252 @@
+"""Parity of the CUDA layer (through the C ABI) with the CPU oracle.
+
+Small shapes are compared in full; full-size layers on sampled tokens with
+every token's routing checked. Indices and lists bit-exact under the 1e-4
+gap rule, outputs within 2e-3 per token row (max |err| / max |y_ref|)."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_harness import (TOL, HostLayer, S, device_blob, expert_source, lists_check, routing_check, row_errors,
+                         torch_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_layer(h: HostLayer, flags=0, max_tokens=None, y0=None):
+    import torch
+    lib = S()
+    mt = max_tokens or max(h.T, 1)
+    dev = torch_dev()
+    bias_d = None if h.bias is None else torch.from_numpy(h.bias).to(dev)
+    layer = lib.MoELayer(h.d, h.f, h.E, h.k, mt, flags=flags, router_bias=bias_d)
+    xd, Wd, _, blob = h.to_device(layer.desc)
+    y = torch.zeros((h.T, h.d), dtype=torch.float32, device=dev) if y0 is None else torch.from_numpy(y0).to(dev)
+    layer.forward(xd, Wd, blob, y, h.T)
+    layer.check_status()
+    idx, w, off, tl, sl = (a.cpu().numpy() for a in layer.routing(h.T))
+    logits = torch.empty((h.T, h.E), dtype=torch.float32, device=dev)
+    layer.router_logits(xd, Wd, logits, h.T)
+    layer.check_status()
+    out = dict(y=y.cpu().numpy(), idx=idx, w=w, off=off, tl=tl, sl=sl, logits=logits.cpu().numpy())
+    layer.close()
+    return out
+
+
+def check_full(h: HostLayer, g, exact_routing=True):
+    y_ref, idx_ref, w_ref = h.oracle()
+    logits_ref = oracle.router_logits(h.x, h.W, h.bias)
+    scale = np.abs(synth.bf16_bits_to_f32(h.x).astype(np.float64)) @ np.abs(h.W.astype(np.float64)).T
+    if h.bias is not None:
+        scale += np.abs(h.bias)
+    assert np.all(np.abs(g["logits"] - logits_ref) <= 1e-5 * np.maximum(scale, 1.0)), "router logits"
+    exempt, bad = routing_check(logits_ref, h.k, g["idx"])
+    assert not bad, f"routing differs for tokens {bad[:10]}"
+    if exact_routing:
+        assert not exempt.any()
+    lists_check(idx_ref, g["idx"], exempt, h.E, g["off"], g["tl"], g["sl"])
+    ok = ~exempt | np.array([sorted(a) == sorted(b) for a, b in zip(g["idx"], idx_ref)])
+    wrow = np.abs(g["w"] - w_ref).max(axis=1)
+    assert np.all(wrow[ok] <= 1e-5), f"routing weights: {wrow.max():.2e}"
+    err = row_errors(g["y"], y_ref)
+    assert np.all(err[ok] <= TOL), f"max row error {err[ok].max():.3e}"
+    return err
+
+
+@pytest.mark.parametrize("flags", [0, 2], ids=["decode", "prefill"])
+def test_tiny_layer(flags):
+    h = HostLayer(256, 128, 16, 4, 8, seed=0)
+    err = check_full(h, run_layer(h, flags))
+    print(f"tiny flags={flags}: max row err {err.max():.2e}")
+
+
+SHAPES = [
+    # d, f, E, k, T, zipf
+    (256, 128, 16, 4, 1, False),
+    (256, 128, 16, 4, 3, True),
+    (256, 128, 16, 4, 16, False),
+    (128, 128, 4, 4, 5, False),        # k = E
+    (384, 256, 64, 10, 13, True),
+    (256, 256, 64, 10, 17, True),      # first prefill size
+    (512, 128, 64, 4, 130, True),      # ragged tiles
+    (256, 384, 32, 8, 300, True),
+    (128, 256, 16, 2, 1000, True),     # large groups, several 128/256 tiles per expert
+]
+
+
+@pytest.mark.parametrize("d,f,E,k,T,zipf", SHAPES)
+def test_shapes(d, f, E, k, T, zipf):
+    h = HostLayer(d, f, E, k, T, seed=d + f + E + k + T, zipf=zipf)
+    for flags in ([0, 2] if T <= 16 else [0]):
+        check_full(h, run_layer(h, flags), exact_routing=False)
+
+
+def test_accumulate_flag():
+    h = HostLayer(256, 128, 16, 4, 6, seed=11)
+    y0 = np.random.default_rng(3).standard_normal((6, 256)).astype(np.float32)
+    y_ref, _, _ = h.oracle()
+    for flags in (1, 3):  # ACCUMULATE, ACCUMULATE | FORCE_PREFILL
+        g = run_layer(h, flags, y0=y0.copy())
+        err = row_errors(g["y"] - y0, y_ref)
+        assert err.max() <= TOL
+
+
+def test_generated_ties():
+    """Duplicated router rows, all-zero rows and equal biases: exact ties go
+    to the lower expert index."""
+    d, f, E, k, T = 256, 128, 16, 4, 12
+    h = HostLayer(d, f, E, k, T, seed=21)
+    W = h.W.copy()
+    W[5] = W[2]
+    W[9] = W[2]
+    W[12] = 0.0
+    W[13] = 0.0
+    W[14] = W[3]
+    bias = np.zeros(E, np.float32)
+    bias[[2, 5, 9]] = 3.0      # the duplicated rows win and tie exactly
+    bias[[12, 13]] = 2.5
+    h2 = HostLayer(d, f, E, k, T, x=h.x, W=W, bias=bias, experts=h.experts)
+    for flags in (0, 2):
+        g = run_layer(h2, flags)
+        check_full(h2, g, exact_routing=False)
+        for t in range(T):
+            sel = list(g["idx"][t])
+            for a, b in ((2, 5), (5, 9), (2, 9), (12, 13), (3, 14)):
+                if b in sel:
+                    assert a in sel and sel.index(a) < sel.index(b), f"tie rule, token {t}: {sel}"
+
+
+def test_zero_scale_and_identity_experts():
+    d, f, E, k, T = 256, 128, 4, 2, 6
+    ident = pins_identity(d, f)
+    zero = dict(ident)
+    zero["gate_scales"] = np.zeros_like(ident["gate_scales"])
+    zero["up_scales"] = np.zeros_like(ident["up_scales"])
+    zero["down_scales"] = np.zeros_like(ident["down_scales"])
+    rng = np.random.default_rng(6)
+    xf = np.zeros((T, d), np.float32)
+    xf[:, ::32] = rng.standard_normal((T, d // 32)) * 2
+    x = synth.f32_to_bf16_bits(xf)
+    W = (rng.standard_normal((E, d)) * 0.3).astype(np.float32)
+    h = HostLayer(d, f, E, k, T, x=x, W=W, experts=[ident, zero, ident, zero])
+    for flags in (0, 2):
+        check_full(h, run_layer(h, flags), exact_routing=False)
+
+
+def pins_identity(d, f):
+    import pins_lib
+    return pins_lib.identity_like_expert(d, f, 1.0)
+
+
+@pytest.mark.parametrize("n", [15, 16, 17, 127, 128, 129, 255, 256, 257])
+def test_group_at_tile_boundaries(n):
+    """Expert 1 gets exactly n tokens (k = 1), the rest go to expert 0."""
+    d, f, E, k = 256, 128, 8, 1
+    T = 300
+    rng = np.random.default_rng(n)
+    xf = (rng.standard_normal((T, d)) * 0.01).astype(np.float32)
+    g = np.zeros(T, int)
+    g[rng.permutation(T)[:n]] = 1
+    xf[np.arange(T), g] = 4.0
+    W = np.zeros((E, d), np.float32)
+    W[np.arange(E), np.arange(E)] = 1.0
+    h = HostLayer(d, f, E, k, T, seed=n, x=synth.f32_to_bf16_bits(xf), W=W)
+    out = run_layer(h, 0)
+    assert out["off"][2] - out["off"][1] == n
+    check_full(h, out, exact_routing=False)
+
+
+def test_single_expert_takes_all():
+    d, f, E, k, T = 256, 128, 16, 1, 40
+    h = HostLayer(d, f, E, k, T, seed=31)
+    bias = np.zeros(E, np.float32)
+    bias[7] = 100.0
+    h.bias = bias
+    for flags in (0, 2) if T <= 16 else (0,):
+        out = run_layer(h, flags)
+        assert np.all(out["idx"][:, 0] == 7)
+        check_full(h, out)
+
+
+def test_zero_tokens_and_too_many():
+    import torch
+    lib = S()
+    layer = lib.MoELayer(256, 128, 16, 4, 8)
+    dev = torch_dev()
+    x = torch.zeros((9, 256), dtype=torch.bfloat16, device=dev)
+    W = torch.zeros((16, 256), dtype=torch.float32, device=dev)
+    blob = torch.zeros(16 * 30720, dtype=torch.uint8, device=dev)
+    y = torch.full((9, 256), 7.0, device=dev)
+    layer.forward(x, W, blob, y, 0)  # no-op
+    assert torch.all(y == 7.0)
+    with pytest.raises(lib.StrataError) as ei:
+        layer.forward(x, W, blob, y, 9)
+    assert ei.value.status == lib.STRATA_ERR_TOO_MANY_TOKENS
+    with pytest.raises(lib.StrataError) as ei:
+        layer.forward(x, W, blob[1:], y, 4)
+    assert ei.value.status == lib.STRATA_ERR_BAD_BLOB
+    layer.close()
+
+
+# ---------------------------------------------------------------- full size
+
+
+def full_size_check(w: synth.Workload, T: int, flags: int, sample: int, layer_idx: int = 0):
+    import torch
+    lib = S()
+    dev = torch_dev()
+    x = synth.gen_x_bf16(w.seed, T, w.d)
+    W = synth.gen_router_w(w.seed, layer_idx, w.E, w.d)
+    bias = synth.router_bias(w, layer_idx)
+    bias_d = None if bias is None else torch.from_numpy(bias).to(dev)
+    layer = lib.MoELayer(w.d, w.f, w.E, w.k, T, flags=flags, router_bias=bias_d)
+    blob = device_blob(w, layer_idx, layer.desc)
+    xd = torch.from_numpy(x.view(np.int16)).to(dev)
+    Wd = torch.from_numpy(W).to(dev)
+    y = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
+    layer.forward(xd, Wd, blob, y, T)
+    layer.check_status()
+    idx, wg, off, tl, sl = (a.cpu().numpy() for a in layer.routing(T))
+    yg = y.cpu().numpy()
+    layer.close()
+    del blob
+    torch.cuda.empty_cache()
+
+    route = oracle.route_layer(x, W, bias, w.k)
+    exempt, bad = routing_check(route["logits"], w.k, idx)
+    assert not bad, f"routing differs for tokens {bad[:10]}"
+    lists_check(route["idx"], idx, exempt, w.E, off, tl, sl)
+    rng = np.random.default_rng(T)
+    cand = np.nonzero(~exempt)[0]
+    toks = np.sort(rng.choice(cand, size=min(sample, cand.size), replace=False))
+    y_ref = oracle.layer_outputs(x, route, toks, expert_source(w, layer_idx))
+    err = row_errors(yg[toks], y_ref)
+    assert err.max() <= TOL, f"max row error {err.max():.3e}"
+    return err.max(), int(exempt.sum())
+
+
+def test_decode_layer_full_size():
+    """One token, 512 experts, top-10, uniform routing (d=2048, f=768)."""
+    e, nex = full_size_check(synth.WORKLOADS["decode"], 1, 0, 1)
+    print(f"decode T=1: max row err {e:.2e}")
+
+
+@pytest.mark.parametrize("T", [2, 4, 7, 16])
+def test_verify_layer_full_size(T):
+    """Decode/verify sizes with the Zipf(1.1) prior, all tokens checked."""
+    e, nex = full_size_check(synth.WORKLOADS["verify4"], T, 0, T)
+    print(f"verify T={T}: max row err {e:.2e}, exempt {nex}")
+
+
+@pytest.mark.parametrize("T", [4, 300])
+def test_prefill_path_full_size_small_T(T):
+    e, nex = full_size_check(synth.WORKLOADS["prefill"], T, 2, min(T, 24))
+    print(f"prefill-path T={T}: max row err {e:.2e}, exempt {nex}")
+
+
+def test_prefill_layer_8192_sampled():
+    """8,192-token chunk, Zipf routing: every token's routing and lists,
+    expert outputs on 48 sampled tokens."""
+    e, nex = full_size_check(synth.WORKLOADS["prefill"], 8192, 0, 48)
+    print(f"prefill T=8192: max row err {e:.2e}, exempt {nex}")
