@@ -155,7 +155,7 @@ def run_strata(args, world, rank, local):
     stacked = w.layers > 1
     T = w.T
     chunk = min(T, w.chunk)
-    copies = 8 if w.name == "decode" else (w.layers if stacked else 1)
+    copies = args.copies if w.name == "decode" else (w.layers if stacked else 1)
     ntok = 64 if w.name == "decode" else 1
 
     # inputs (each rank holds its own replica)
@@ -231,6 +231,7 @@ def run_strata(args, world, rank, local):
     ms_step = ms / args.steps
     tokens = T * args.steps * world
     value = tokens / (ms / 1e3)
+    print(f"# timed region: {ms_step * 1e3:.2f} us/step, {value:.1f} tokens/s", file=sys.stderr, flush=True)
 
     # stage timing of the dominant kernel (separate pass, events around it)
     dom = stage_timing(S, w, handles, handle, layers, xs, y, x_res, T, copies, ntok, stacked)
@@ -251,7 +252,7 @@ def run_strata(args, world, rank, local):
         "data": "synthetic (seeded; random-init 2-bit experts)",
         "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
                    "tokens_per_step": T, "layers": w.layers, "routing": "zipf1.1" if w.zipf else "uniform",
-                   "l2": ("inputs larger than L2: 8 seeded layer copies (6.0 GB) and 64 token vectors rotated"
+                   "l2": (f"inputs larger than L2: {copies} seeded layer copies ({copies * 0.755:.1f} GB) and 64 token vectors rotated"
                           if w.name == "decode" else "inputs larger than L2 (0.75 GB per layer)"),
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roof,
@@ -460,6 +461,7 @@ def main():
     ap.add_argument("--impl", default="strata", choices=["strata", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copies", type=int, default=8, help="decode: seeded layer copies rotated (8 = 6 GB)")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {"decode": 64 * 1024, "verify4": 200, "verify16": 100, "prefill": 200,

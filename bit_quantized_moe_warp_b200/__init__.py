@@ -12,7 +12,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstrata_moe.so")
+# STRATA_MOE_LIB selects another build of the same library (e.g. an instrumented one)
+LIB_PATH = os.environ.get("STRATA_MOE_LIB") or os.path.join(_HERE, "libstrata_moe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_quantized_moe_warp_b200.build` "

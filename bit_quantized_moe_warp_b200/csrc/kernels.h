@@ -24,13 +24,14 @@ struct Workspace {
     int32_t *pair_of;     // [T * k]   (t, j) -> index in the sorted pair list
     int32_t *blk_counts;  // [nblk * E] per 256-token block (prefill lists)
     int32_t *act;         // [E] active experts (decode path)
-    float *gu_part;       // [KS * Pd * 2 * f]   decode gate/up partial sums
-    float *o_part;        // [KSD * Pd * d]      decode down partial outputs
+    float *gu_part;       // [KS * Pd * 2 * f]   fused decode: gate/up partial sums
+    float *lpart;         // [16 * E * 4]        fused decode: router partial sums
     void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill)
     void *hbuf;           // fp16 [T*k * f]       SwiGLU outputs (prefill)
     int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
     int4 *tiles2;         // down GEMM tiles
     void *xn;             // bf16 [T * d]         stack: normalised input
+    uint32_t *sync;       // [2 + E] fused decode: grid barrier, exit count, per-expert gate/up counters
 };
 
 // meta[] slots
@@ -38,8 +39,7 @@ enum { META_N_ACTIVE = 0, META_N_TILES1 = 1, META_N_TILES2 = 2, META_N_TOKENS = 
 
 constexpr int kRouteBlock = 256;      // tokens per block of the prefill lists
 constexpr int kDecMaxT = 16;          // largest token count of the streaming path
-constexpr int kDecKS = 4;             // decode gate/up K splits (max)
-constexpr int kDecKSD = 2;            // decode down K splits
+constexpr int kDecKS = 4;             // fused decode gate/up K splits (max)
 constexpr int kGemm1N = 128;          // gate/up GEMM: max tokens per tile
 constexpr int kGemm2N = 256;          // down GEMM: max tokens per tile
 
@@ -56,15 +56,16 @@ void launch_router_gemv(const void *x, const float *W, const float *bias, float 
                         cudaStream_t st);
 void launch_router_gemm(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
                         cudaStream_t st);
-void launch_route_small(const Workspace &ws, int T, const Shape &s, cudaStream_t st);
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
                         cudaStream_t st);
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st);
 
-// --- decode experts (T <= 16)
-// stage_ev (nullable): [2] / [3] are recorded around the gate/up kernel
-void launch_decode_experts(const Workspace &ws, const void *x, const uint8_t *blob, float *y, bool accumulate,
-                           int T, const Shape &s, int num_sms, cudaStream_t st, cudaEvent_t *stage_ev);
+// --- fused decode layer (T <= 16, one cooperative launch)
+bool decode_fused_supported(const Shape &s, int T, int max_smem);
+cudaError_t init_fused_attributes(int max_smem);
+cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float *W, const float *bias,
+                                const uint8_t *blob, float *y, bool accumulate, bool rms, float eps, int T,
+                                const Shape &s, int num_sms, int max_smem, cudaStream_t st, cudaEvent_t *ev);
 
 // --- prefill experts (tensor cores)
 void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
@@ -79,6 +80,16 @@ void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int
 void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st);
 
 size_t expert_bytes(const Shape &s);
+
+// Allow `kernel` the largest dynamic shared memory the device grants a block
+// (max_total, the opt-in limit) minus its static shared memory.
+template <typename Kernel>
+inline cudaError_t set_max_dynamic_smem(Kernel kernel, int max_total) {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_total - (int)a.sharedSizeBytes);
+}
 size_t down_section_offset(const Shape &s);
 
 }  // namespace strata

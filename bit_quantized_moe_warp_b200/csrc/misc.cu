@@ -34,8 +34,9 @@ void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cud
 }
 
 // ------------------------------------------------------------ packer
-// One thread per (tile, row): 64 codes -> four words (column c in word c/16
-// at bit 16*(c%2) + 2*((c%16)/2)), then the row's two block scales.
+// One thread per (tile, row): 64 codes -> four words (column
+// c = 16j + 8s + 2t + h in word t at bit 16h + 8s + 6 - 2j), then the row's
+// two block scales.
 __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales, int rows, int K,
                               uint8_t *__restrict__ dst, size_t tile_stride) {
     const int slices = K / 64;
@@ -51,7 +52,7 @@ __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t 
 #pragma unroll 4
     for (int c = 0; c < 64; ++c) {
         const uint32_t v = cr[c] & 3u;
-        w[c >> 4] |= v << (16 * (c & 1) + 2 * ((c & 15) >> 1));
+        w[(c & 7) >> 1] |= v << (16 * (c & 1) + 8 * ((c >> 3) & 1) + 6 - 2 * (c >> 4));
     }
     uint8_t *t = dst + (size_t)tile * tile_stride;
     *reinterpret_cast<uint4 *>(t + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);

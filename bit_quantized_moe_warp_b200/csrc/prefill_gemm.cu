@@ -243,15 +243,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
                 uint8_t *arow = A_at(st, mat) + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 8; ++c) {  // output chunk c: columns 8c .. 8c+7
                     if (c < c_lo || c >= c_hi) continue;
-                    const uint32_t w = words[c >> 1];
                     const __half2 sc = (c < 4) ? sh0 : sh1;
+                    // columns 8c + 2t, 8c + 2t + 1 sit in word t, halves 0/1, at bit
+                    // 8 (c & 1) + 6 - 2 (c >> 1); bring them to bits 1-2 of each half
+                    const int pos = 8 * (c & 1) + 6 - 2 * (c >> 1);
                     uint32_t out[4];
 #pragma unroll
                     for (int pr = 0; pr < 4; ++pr) {
-                        const int mp = 4 * (c & 1) + pr;
-                        uint32_t v = (mp == 0) ? (w << 1) : (w >> (2 * mp - 1));
+                        const uint32_t w = words[pr];
+                        uint32_t v = (pos == 0) ? (w << 1) : (w >> (pos - 1));
                         v = (v & 0x00060006u) | 0x64006400u;  // fp16 1024 + 2c in both halves
                         __half2 h = *reinterpret_cast<__half2 *>(&v);
                         h = __hmul2(__hsub2(h, k1027), sc);    // (2c - 3) * s/2 = (c - 1.5) s
@@ -279,11 +281,12 @@ static void launch_gemm(const TmaMaps &maps, const GemmArgs &a, int num_sms, cud
     k_expert_gemm<MODE><<<num_sms, kGemmThreads, L::SMEM, st>>>(maps, a);
 }
 
-void init_gemm_attributes(int max_smem) {
-    static_assert(GLayout<0>::SMEM <= 232448 && GLayout<1>::SMEM <= 232448, "shared memory budget");
-    (void)max_smem;
-    cudaFuncSetAttribute(k_expert_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<0>::SMEM);
-    cudaFuncSetAttribute(k_expert_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<1>::SMEM);
+cudaError_t init_gemm_attributes(int max_smem) {
+    if ((int)GLayout<0>::SMEM > max_smem || (int)GLayout<1>::SMEM > max_smem) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)GLayout<0>::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_expert_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<1>::SMEM);
 }
 
 void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,

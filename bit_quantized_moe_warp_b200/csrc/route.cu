@@ -165,64 +165,6 @@ __device__ void warp_topk(const float *__restrict__ lrow, int E, int k, int *sel
     }
 }
 
-// ------------------------------------------------------------ small lists
-// Decode sizes (T <= 16): one block does top-k for every token, counts,
-// exclusive scan, stable (ascending token) scatter of the (token, slot)
-// pairs and the list of active experts.
-__global__ void __launch_bounds__(512) k_route_small(Workspace ws, int T, int E, int k) {
-    __shared__ int s_idx[16 * 32];
-    __shared__ float s_w[16 * 32];
-    __shared__ int s_cnt[1024];
-    __shared__ int s_off[1025];
-    __shared__ int s_act[1024];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp < T) {
-        warp_topk(ws.logits + (size_t)warp * E, E, k, s_idx + warp * 32, s_w + warp * 32);
-        __syncwarp();
-        if (lane < k) {
-            ws.topk_idx[warp * k + lane] = s_idx[warp * 32 + lane];
-            ws.topk_w[warp * k + lane] = s_w[warp * 32 + lane];
-        }
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int t = 0; t < T; ++t)
-            for (int j = 0; j < k; ++j) c += (s_idx[t * 32 + j] == e);
-        s_cnt[e] = c;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {  // E <= 1024: serial scan is a few microseconds at most
-        int run = 0, na = 0;
-        for (int e = 0; e < E; ++e) {
-            s_off[e] = run;
-            run += s_cnt[e];
-            if (s_cnt[e]) s_act[na++] = e;
-        }
-        s_off[E] = run;
-        ws.meta[META_N_ACTIVE] = na;
-        ws.meta[META_N_TOKENS] = T;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) ws.offsets[e] = s_off[e];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        ws.counts[e] = s_cnt[e];
-        ws.act[e] = s_act[e];  // entries past n_active are stale, never read
-    }
-    for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
-        int t = p / k, j = p % k;
-        int e = s_idx[t * 32 + j];
-        int rank = 0;
-        for (int t2 = 0; t2 < t; ++t2)
-            for (int j2 = 0; j2 < k; ++j2) rank += (s_idx[t2 * 32 + j2] == e);
-        int pos = s_off[e] + rank;
-        ws.token_list[pos] = t;
-        ws.pair_slot[pos] = j;
-        ws.pair_w[pos] = s_w[t * 32 + j];
-        ws.pair_of[p] = pos;
-    }
-}
-
 // ------------------------------------------------------------ large lists
 // Prefill sizes. (1) top-k per token, per-256-token-block expert counts.
 __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E, int k) {
@@ -381,10 +323,6 @@ void launch_router_gemm(const void *x, const float *W, const float *bias, float 
                         cudaStream_t st) {
     dim3 grid((s.E + 63) / 64, (T + 63) / 64), block(256);
     k_router_gemm<<<grid, block, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), W, bias, logits, T, s.d, s.E);
-}
-
-void launch_route_small(const Workspace &ws, int T, const Shape &s, cudaStream_t st) {
-    k_route_small<<<1, 512, 0, st>>>(ws, T, s.E, s.k);
 }
 
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,

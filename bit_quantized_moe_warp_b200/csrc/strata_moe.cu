@@ -91,7 +91,7 @@ static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
-    size_t off[20];
+    size_t off[21];
     size_t total;
     int max_tiles1, max_tiles2;
 };
@@ -105,7 +105,7 @@ static Plan plan_workspace(const strata_moe_desc *d) {
     Plan p{};
     p.max_tiles1 = (int)((P + kGemm1N - 1) / kGemm1N + E);
     p.max_tiles2 = (int)((P + kGemm2N - 1) / kGemm2N + E);
-    const size_t sz[20] = {
+    const size_t sz[21] = {
         256,                                      // 0 status
         64 * 4,                                   // 1 meta
         T * E * 4,                                // 2 logits
@@ -120,15 +120,16 @@ static Plan plan_workspace(const strata_moe_desc *d) {
         nblk * E * 4,                             // 11 blk_counts
         E * 4,                                    // 12 act
         (size_t)kDecKS * Pd * 2 * s.f * 4,        // 13 gu_part
-        (size_t)kDecKSD * Pd * s.d * 4,           // 14 o_part
+        (size_t)kDecMaxT * E * 4 * 4,             // 14 lpart
         P * (size_t)s.d * 2,                      // 15 xp
         P * (size_t)s.f * 2,                      // 16 hbuf
         (size_t)p.max_tiles1 * 16,                // 17 tiles1
         (size_t)p.max_tiles2 * 16,                // 18 tiles2
         T * (size_t)s.d * 2,                      // 19 xn
+        (2 + E) * 4,                              // 20 sync
     };
     size_t o = 0;
-    for (int i = 0; i < 20; ++i) {
+    for (int i = 0; i < 21; ++i) {
         p.off[i] = o;
         o += (sz[i] + 255) & ~(size_t)255;
     }
@@ -152,12 +153,13 @@ static Workspace carve(uint8_t *base, const Plan &p) {
     w.blk_counts = reinterpret_cast<int32_t *>(base + p.off[11]);
     w.act = reinterpret_cast<int32_t *>(base + p.off[12]);
     w.gu_part = reinterpret_cast<float *>(base + p.off[13]);
-    w.o_part = reinterpret_cast<float *>(base + p.off[14]);
+    w.lpart = reinterpret_cast<float *>(base + p.off[14]);
     w.xp = base + p.off[15];
     w.hbuf = base + p.off[16];
     w.tiles1 = reinterpret_cast<int4 *>(base + p.off[17]);
     w.tiles2 = reinterpret_cast<int4 *>(base + p.off[18]);
     w.xn = base + p.off[19];
+    w.sync = reinterpret_cast<uint32_t *>(base + p.off[20]);
     return w;
 }
 
@@ -198,13 +200,13 @@ static strata_status make_maps(TmaMaps &m, void *base, size_t rows, int K) {
 }
 
 namespace strata {
-void init_decode_attributes(int max_smem);
-void init_gemm_attributes(int max_smem);
-static void init_kernel_attributes(int device) {
+cudaError_t init_gemm_attributes(int max_smem);
+static cudaError_t init_kernel_attributes(int device) {
     int max_smem = 0;
-    cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
-    init_decode_attributes(max_smem);
-    init_gemm_attributes(max_smem);
+    cudaError_t e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    if (e == cudaSuccess) e = init_gemm_attributes(max_smem);
+    if (e == cudaSuccess) e = init_fused_attributes(max_smem);
+    return e;
 }
 }  // namespace strata
 
@@ -216,6 +218,7 @@ struct StackGraph {
 
 struct strata_moe_layer_s {
     strata_moe_desc desc;
+    cudaStream_t capture_stream;  // private stream the stack graph is captured on
     Shape shape;
     int device;
     int num_sms;
@@ -224,13 +227,15 @@ struct strata_moe_layer_s {
     Plan plan;
     Workspace ws;
     TmaMaps maps1, maps2;
+    bool fused_ok;   // the one-launch streaming layer fits this shape
+    int max_smem;
     StackGraph graph;
     cudaEvent_t stage_ev[5];
     bool stage_on;
 };
 
 static void stage_mark(strata_moe_layer L, int i, cudaStream_t st) {
-    if (L->stage_on) cudaEventRecord(L->stage_ev[i], st);
+    if (L->stage_on) cudaEventRecordWithFlags(L->stage_ev[i], st, cudaEventRecordExternal);
 }
 
 extern "C" strata_status strata_moe_set_stage_events(strata_moe_layer L, void *const *events, int32_t n) {
@@ -323,11 +328,23 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
         delete L;
         return s;
     }
-    init_kernel_attributes(L->device);
-    if ((s = check_launch("kernel attributes")) != STRATA_OK) {
+    {
+        int max_smem = 0;
+        cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, L->device);
+        const int Tw = desc->max_tokens < kDecMaxT ? desc->max_tokens : kDecMaxT;
+        L->fused_ok = decode_fused_supported(L->shape, Tw, max_smem);
+        L->max_smem = max_smem;
+    }
+    if (cudaMemset(L->ws.sync, 0, (size_t)(2 + L->shape.E) * 4) != cudaSuccess) {
         if (L->owns_ws) cudaFree(L->ws_mem);
         delete L;
-        return s;
+        return fail(STRATA_ERR_CUDA, "workspace clear failed");
+    }
+    if (cudaError_t e = init_kernel_attributes(L->device)) {
+        cudaGetLastError();
+        if (L->owns_ws) cudaFree(L->ws_mem);
+        delete L;
+        return fail(STRATA_ERR_CUDA, "kernel attribute set-up failed: %s", cudaGetErrorString(e));
     }
     *out = L;
     return STRATA_OK;
@@ -336,6 +353,7 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
 extern "C" strata_status strata_moe_layer_destroy(strata_moe_layer L) {
     if (!L) return STRATA_OK;
     if (L->graph.exec) cudaGraphExecDestroy(L->graph.exec);
+    if (L->capture_stream) cudaStreamDestroy(L->capture_stream);
     if (L->owns_ws) cudaFree(L->ws_mem);
     delete L;
     return STRATA_OK;
@@ -353,34 +371,28 @@ static strata_status check_layer(strata_moe_layer L, int32_t T, bool layer_call)
 }
 
 static bool use_decode(strata_moe_layer L, int T) {
-    return T <= kDecMaxT && !(L->desc.flags & STRATA_FORCE_PREFILL);
+    return T <= kDecMaxT && L->fused_ok && !(L->desc.flags & STRATA_FORCE_PREFILL);
 }
 
 static strata_status route_impl(strata_moe_layer L, const void *x, const float *W, const float *bias, int T,
                                 cudaStream_t st) {
-    if (use_decode(L, T)) {
+    if (T <= kDecMaxT)
         launch_router_gemv(x, W, bias, L->ws.logits, T, L->shape, st);
-        launch_route_small(L->ws, T, L->shape, st);
-    } else {
+    else
         launch_router_gemm(x, W, bias, L->ws.logits, T, L->shape, st);
-        launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st);
-    }
+    launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st);
     return check_launch("routing kernels");
 }
 
 static strata_status experts_impl(strata_moe_layer L, const void *x, const void *blob, float *y, int T, bool acc,
                                   cudaStream_t st) {
     const uint8_t *b = static_cast<const uint8_t *>(blob);
-    if (use_decode(L, T)) {
-        launch_decode_experts(L->ws, x, b, y, acc, T, L->shape, L->num_sms, st, L->stage_on ? L->stage_ev : nullptr);
-    } else {
-        if (!acc) CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)T * L->shape.d * sizeof(float), st));
-        launch_gather_xp(L->ws, x, T, L->shape, st);
-        stage_mark(L, 2, st);
-        launch_expert_gemm1(L->ws, b, L->maps1, L->plan.max_tiles1, L->shape, L->num_sms, st);
-        stage_mark(L, 3, st);
-        launch_expert_gemm2(L->ws, b, y, L->maps2, L->plan.max_tiles2, L->shape, L->num_sms, st);
-    }
+    if (!acc) CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)T * L->shape.d * sizeof(float), st));
+    launch_gather_xp(L->ws, x, T, L->shape, st);
+    stage_mark(L, 2, st);
+    launch_expert_gemm1(L->ws, b, L->maps1, L->plan.max_tiles1, L->shape, L->num_sms, st);
+    stage_mark(L, 3, st);
+    launch_expert_gemm2(L->ws, b, y, L->maps2, L->plan.max_tiles2, L->shape, L->num_sms, st);
     return check_launch("expert kernels");
 }
 
@@ -399,6 +411,15 @@ extern "C" strata_status strata_moe_forward(strata_moe_layer L, const void *x, c
     if (T == 0) return STRATA_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     stage_mark(L, 0, st);
+    if (use_decode(L, T)) {
+        stage_mark(L, 1, st);
+        cudaError_t e = launch_decode_fused(L->ws, x, W, L->desc.router_bias, static_cast<const uint8_t *>(blob), y,
+                                            (L->desc.flags & STRATA_ACCUMULATE) != 0, false, 0.f, T, L->shape,
+                                            L->num_sms, L->max_smem, st, L->stage_on ? L->stage_ev : nullptr);
+        stage_mark(L, 4, st);
+        if (e != cudaSuccess) return fail(STRATA_ERR_CUDA, "fused decode launch: %s", cudaGetErrorString(e));
+        return check_launch("fused decode kernel");
+    }
     if ((s = route_impl(L, x, W, L->desc.router_bias, T, st)) != STRATA_OK) return s;
     stage_mark(L, 1, st);
     s = experts_impl(L, x, blob, y, T, (L->desc.flags & STRATA_ACCUMULATE) != 0, st);
@@ -415,7 +436,7 @@ extern "C" strata_status strata_moe_router_logits(strata_moe_layer L, const void
         return fail(STRATA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
     if (T == 0) return STRATA_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (use_decode(L, T))
+    if (T <= kDecMaxT)
         launch_router_gemv(x, W, L->desc.router_bias, logits, T, L->shape, st);
     else
         launch_router_gemm(x, W, L->desc.router_bias, logits, T, L->shape, st);
@@ -481,6 +502,15 @@ static strata_status stack_enqueue(strata_moe_layer L, int n_layers, const float
                                    const float *const *bias, const void *const *blobs, float *x, int T, float eps,
                                    cudaStream_t st) {
     strata_status s;
+    if (use_decode(L, T)) {  // RMSNorm, routing and experts in one launch per layer
+        for (int l = 0; l < n_layers; ++l) {
+            const float *b = bias ? bias[l] : nullptr;
+            cudaError_t e = launch_decode_fused(L->ws, x, W[l], b, static_cast<const uint8_t *>(blobs[l]), x, true,
+                                                true, eps, T, L->shape, L->num_sms, L->max_smem, st, nullptr);
+            if (e != cudaSuccess) return fail(STRATA_ERR_CUDA, "fused decode launch: %s", cudaGetErrorString(e));
+        }
+        return check_launch("fused decode kernels");
+    }
     for (int l = 0; l < n_layers; ++l) {
         launch_rmsnorm_bf16(x, L->ws.xn, T, L->shape.d, eps, st);
         const float *b = bias ? bias[l] : nullptr;
@@ -535,10 +565,14 @@ extern "C" strata_status strata_moe_stack_forward(strata_moe_layer L, int32_t n_
             cudaGraphExecDestroy(L->graph.exec);
             L->graph.exec = nullptr;
         }
-        CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-        s = stack_enqueue(L, n_layers, W, bias, blobs, x, T, eps, st);
+        // capture on the library's own stream (the caller's may be the legacy
+        // default stream, which cannot be captured); the graph is launched on
+        // the caller's stream
+        if (!L->capture_stream) CUDA_TRY(cudaStreamCreateWithFlags(&L->capture_stream, cudaStreamNonBlocking));
+        CUDA_TRY(cudaStreamBeginCapture(L->capture_stream, cudaStreamCaptureModeThreadLocal));
+        s = stack_enqueue(L, n_layers, W, bias, blobs, x, T, eps, L->capture_stream);
         cudaGraph_t g = nullptr;
-        cudaError_t ce = cudaStreamEndCapture(st, &g);
+        cudaError_t ce = cudaStreamEndCapture(L->capture_stream, &g);
         if (s != STRATA_OK) {
             if (g) cudaGraphDestroy(g);
             return s;
@@ -562,7 +596,10 @@ extern "C" strata_status strata_moe_check_status(strata_moe_layer L) {
     uint32_t w = 0;
     CUDA_TRY(cudaMemcpy(&w, L->ws.status, 4, cudaMemcpyDeviceToHost));
     CUDA_TRY(cudaMemset(L->ws.status, 0, 4));
-    if (w & kStatusTimeout) return fail(STRATA_ERR_TIMEOUT, "a device wait exceeded its time limit");
+    if (w & kStatusTimeout) {
+        cudaMemset(L->ws.sync, 0, (size_t)(2 + L->shape.E) * 4);  // counters of an unwound launch
+        return fail(STRATA_ERR_TIMEOUT, "a device wait exceeded its time limit");
+    }
     return STRATA_OK;
 }
 
@@ -596,8 +633,9 @@ static void pack_matrix_host(const uint8_t *codes, const uint16_t *scales, int r
             for (int i = 0; i < 128; ++i) {
                 const int r = p * 128 + i;
                 uint32_t w[4] = {0, 0, 0, 0};
-                for (int c = 0; c < 64; ++c)
-                    w[c / 16] |= (uint32_t)(codes[(size_t)r * K + 64 * s + c] & 3u) << (16 * (c % 2) + 2 * ((c % 16) / 2));
+                for (int c = 0; c < 64; ++c)  // c = 16j + 8s + 2t + h -> word t, bit 16h + 8s + 6 - 2j
+                    w[(c % 8) / 2] |= (uint32_t)(codes[(size_t)r * K + 64 * s + c] & 3u)
+                                      << (16 * (c % 2) + 8 * ((c / 8) % 2) + 6 - 2 * (c / 16));
                 for (int q = 0; q < 4; ++q)
                     for (int b = 0; b < 4; ++b) t[16 * i + 4 * q + b] = (uint8_t)(w[q] >> (8 * b));
                 for (int b = 0; b < 2; ++b) {

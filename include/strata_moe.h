@@ -65,11 +65,15 @@ typedef enum {
  * A matrix [R x K] (R % 128 == 0, K % 64 == 0) is a sequence of tiles, one
  * per (128-row panel p, 64-column slice s); a tile is 2560 bytes:
  *   bytes [0, 2048):   codes, row i (0..127) at bytes 16i..16i+15, as four
- *                      little-endian uint32 words; column c (0..63) of the
- *                      tile lives in word c/16 at bit 16*(c%2) + 2*((c%16)/2)
- *                      (even columns in the low halves, odd columns in the
- *                      high halves, so one shift and mask yields two codes
- *                      for adjacent columns);
+ *                      little-endian uint32 words W0..W3; column c (0..63)
+ *                      of the tile, written c = 16j + 8s + 2t + h (j < 4,
+ *                      s < 2, t < 4, h < 2), lives in word Wt at bit
+ *                      16h + 8s + 6 - 2j. Word t thus holds exactly the 16
+ *                      codes that lane t of a 4-lane group needs for the
+ *                      row in the warp-level 16x8x16 MMA fragment layout
+ *                      (columns 2t, 2t+1, 2t+8, 2t+9 of each 16-column
+ *                      step), and one mask per register extracts the two
+ *                      codes of a column pair without a shift;
  *   bytes [2048, 2560): scales, row i at 2048+4i: fp16 (little-endian) of
  *                      block 2s, then of block 2s+1.
  * Every tile is a multiple of 16 bytes, so tiles serve 128-bit loads and

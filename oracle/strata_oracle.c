@@ -102,9 +102,9 @@ void oracle_dequant(int rows, int K, const uint8_t *codes, const uint16_t *scale
 /* Unpack one matrix of the tiled blob written by the library's packer, from
  * the layout the library's header documents (128-row x 64-column tiles of
  * 2560 bytes; inside a tile, row i's 64 codes occupy bytes 16i..16i+15 as four
- * little-endian 32-bit words; column c of the tile sits in word c/16 at bit
- * 16*(c%2) + 2*((c%16)/2); the row's two fp16 scales follow at byte
- * 2048 + 4i). Tile t starts at byte t * tile_stride (2560 for a lone matrix;
+ * little-endian 32-bit words W0..W3; column c = 16j + 8s + 2t + h of the tile
+ * sits in word Wt at bit 16h + 8s + 6 - 2j; the row's two fp16 scales follow
+ * at byte 2048 + 4i). Tile t starts at byte t * tile_stride (2560 for a lone matrix;
  * 5120 for the interleaved gate/up tiles of an expert). Returns one code per
  * byte and the fp16 scale bits. */
 void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long tile_stride, uint8_t *codes,
@@ -117,10 +117,11 @@ void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long tile_stri
             for (int i = 0; i < 128; ++i) {
                 int r = p * 128 + i;
                 for (int c = 0; c < 64; ++c) {
-                    const uint8_t *wp = tile + 16 * i + 4 * (c / 16);
+                    int j = c / 16, sh = (c / 8) % 2, t = (c % 8) / 2, h = c % 2;
+                    const uint8_t *wp = tile + 16 * i + 4 * t;
                     uint32_t w = (uint32_t)wp[0] | ((uint32_t)wp[1] << 8) |
                                  ((uint32_t)wp[2] << 16) | ((uint32_t)wp[3] << 24);
-                    int bit = 16 * (c % 2) + 2 * ((c % 16) / 2);
+                    int bit = 16 * h + 8 * sh + 6 - 2 * j;
                     codes[(size_t)r * K + 64 * s + c] = (uint8_t)((w >> bit) & 3u);
                 }
                 for (int b = 0; b < 2; ++b) {

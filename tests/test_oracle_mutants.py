@@ -23,7 +23,8 @@ MUTANTS = [
     ("softmax_no_shift", "p[e] = exp(l[e] - mx);", "p[e] = exp(l[e] - mx) + 1e-3;"),
     ("lists_slot_major", "for (int t = 0; t < T; ++t)\n            for (int j = 0; j < k; ++j)\n                if (idx[(size_t)t * k + j] == e) {",
      "for (int j = 0; j < k; ++j)\n            for (int t = 0; t < T; ++t)\n                if (idx[(size_t)t * k + j] == e) {"),
-    ("unpack_bit", "int bit = 16 * (c % 2) + 2 * ((c % 16) / 2);", "int bit = 2 * (c % 16);"),
+    ("unpack_bit", "int bit = 16 * h + 8 * sh + 6 - 2 * j;", "int bit = 16 * h + 8 * sh + 2 * j;"),
+    ("unpack_word", "const uint8_t *wp = tile + 16 * i + 4 * t;", "const uint8_t *wp = tile + 16 * i + 4 * j;"),
     ("unpack_scale_order", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * (1 - b);"),
     ("rms_no_mean", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
     ("rms_eps_outside", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss / d) + eps;"),
