@@ -64,6 +64,7 @@ _SIGS = {
     "strata_moe_route": (I32, [V, V, V, I32, V]),
     "strata_moe_experts": (I32, [V, V, V, V, I32, V]),
     "strata_moe_get_routing": (I32, [V, V, V, V, V, V, V]),
+    "strata_moe_route_noalloc": (I32, [DP, V, V, I32, V, V, V, V, V, V]),
     "strata_moe_stack_forward": (I32, [V, I32, V, V, V, V, I32, ctypes.c_float, V]),
     "strata_rmsnorm_bf16": (I32, [V, V, I32, I32, ctypes.c_float, V]),
     "strata_moe_set_stage_events": (I32, [V, V, I32]),
@@ -160,6 +161,13 @@ def strata_moe_get_routing(layer, topk_idx=None, topk_w=None, expert_offsets=Non
                            pair_slot=None, stream=None):
     _check(_lib.strata_moe_get_routing(layer, _ptr(topk_idx), _ptr(topk_w), _ptr(expert_offsets),
                                        _ptr(token_list), _ptr(pair_slot), _stream(stream)))
+
+
+def strata_moe_route_noalloc(desc, x, router_w, n_tokens, topk_idx, topk_w, expert_offsets, token_list,
+                             pair_slot, stream=None):
+    _check(_lib.strata_moe_route_noalloc(ctypes.byref(desc), _ptr(x), _ptr(router_w), n_tokens, _ptr(topk_idx),
+                                         _ptr(topk_w), _ptr(expert_offsets), _ptr(token_list), _ptr(pair_slot),
+                                         _stream(stream)))
 
 
 def strata_moe_stack_forward(layer, router_w, router_bias, expert_blobs, x_resid, n_tokens, rms_eps,

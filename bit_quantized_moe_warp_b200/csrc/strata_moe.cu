@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "../../include/strata_moe.h"
+#include "abi_internal.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -86,6 +87,16 @@ static strata_status validate_desc(const strata_moe_desc *d) {
         return fail(STRATA_ERR_INVALID_ARG, "router_bias must be 16-byte aligned");
     return STRATA_OK;
 }
+
+strata_status strata_set_error(strata_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+strata_status strata_check_desc(const strata_moe_desc *desc) { return validate_desc(desc); }
 
 static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_ff, d->n_experts, d->top_k}; }
 

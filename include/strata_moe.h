@@ -175,6 +175,35 @@ strata_status strata_moe_get_routing(strata_moe_layer layer, int32_t *topk_idx, 
                                      int32_t *expert_offsets, int32_t *token_list,
                                      int32_t *pair_slot, strata_stream_t stream);
 
+/* Routing without any allocation, for callers that cannot allocate device
+ * memory when they route (all free memory handed to another allocator, or a
+ * loop that must not call cudaMalloc / cudaFree because they can synchronise
+ * the device). The pages have no counterpart of this call: it is this
+ * library's own interface.
+ *
+ * Computes what strata_moe_route computes for desc (router bias from
+ * desc->router_bias; max_tokens and flags are ignored) and writes it to the
+ * caller's device buffers, laid out as strata_moe_get_routing documents:
+ * topk_idx [T x k], topk_w [T x k], expert_offsets [E + 1],
+ * token_list [T*k], pair_slot [T*k] (all required, 4-byte aligned).
+ * x_bf16 [T x d] and router_w [E x d] as for strata_moe_route (16-byte
+ * aligned).
+ *
+ * Limit: n_tokens <= STRATA_NOALLOC_MAX_TOKENS (16); larger counts return
+ * STRATA_ERR_TOO_MANY_TOKENS. The kernels' scratch is a fixed array of
+ * STRATA_NOALLOC_SCRATCH_BYTES in device memory owned by the library, one per
+ * device, whose address is looked up by the first call on each device (make
+ * that first call before capturing a stream that contains the call). No
+ * scratch word needs to start at zero. Calls on one device share that array:
+ * calls whose device work may overlap race on it, so issue them in order
+ * (e.g. on one stream). Asynchronous on `stream`. */
+#define STRATA_NOALLOC_MAX_TOKENS 16
+#define STRATA_NOALLOC_SCRATCH_BYTES (112 * 1024)
+strata_status strata_moe_route_noalloc(const strata_moe_desc *desc, const void *x_bf16,
+                                       const float *router_w, int32_t n_tokens, int32_t *topk_idx,
+                                       float *topk_w, int32_t *expert_offsets, int32_t *token_list,
+                                       int32_t *pair_slot, strata_stream_t stream);
+
 /* A stack of n_layers layers with the residual recurrence
  *   x <- x + MoE_l(bf16(RMSNorm(x)))   (RMSNorm with unit weights, eps)
  * x_resid [n_tokens x d] fp32 in/out. router_w, router_bias and
