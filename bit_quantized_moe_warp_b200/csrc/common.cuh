@@ -94,6 +94,18 @@ STRATA_DEV void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, u
         : "memory");
 }
 
+// 4-byte asynchronous global -> shared copy (the issuing thread does not
+// wait); cp_async_wait_all() by the same thread waits for its copies.
+STRATA_DEV void cp_async4(void *dst_smem, const void *src_gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+STRATA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Ask L2 to fetch [src, src + bytes) from memory (no completion signal).
+STRATA_DEV void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 2-D tiled tensor copy global -> shared (no multicast).
 STRATA_DEV void tma_load_2d(void *dst_smem, const CUtensorMap *map, int32_t x, int32_t y, uint64_t *bar) {
     asm volatile(

@@ -2,36 +2,33 @@
 // cooperative launch (one CTA per SM).
 //
 // A decode step verifies 1 + up to 3 draft tokens in one 48-layer pass
-// ("Strata：把 125B 大模型塞进 12GB 显卡…", 投机解码); every token uses 10
-// experts (核心思路). At these sizes the layer is bound by the bytes of the
-// selected experts' 2-bit weights, so the kernel keeps that stream busy and
-// pays the routing latency once:
+// ("Strata：把 125B 大模型塞进 12GB 显卡，24,576 个专家在内存与 SSD 之间流动",
+// 再快一截：先猜再验的投机解码); every token uses 10 experts (核心思路). At these
+// sizes the layer is bound by the bytes of the selected experts' 2-bit
+// weights and by the latency of the steps before them, so the kernel pays
+// the routing latency once and then keeps the weight stream busy:
 //
-//   phase 0  every CTA stages x (optionally bf16(RMSNorm) of the fp32
-//            residual, the stack glue), computes the router logits of its
-//            slice of experts (fp32, one fixed reduction order per row) and
-//            zeroes its slice of y; grid barrier.
+//   phase 0  one warp per CTA starts bulk copies of x and of the CTA's slice
+//            of router rows; the other warps zero the CTA's slice of y,
+//            stage x as fp16 (or bf16(RMSNorm) of the fp32 residual, the
+//            stack glue) and compute the router partial sums of their rows
+//            (fp32, one fixed reduction order per row); grid barrier.
 //   phase 1  every CTA reads all logits and computes, redundantly and
-//            identically, the softmax top-k of every token (ties to the lower
-//            expert index), the renormalised weights, the per-expert token
-//            lists and the active experts (CTA 0 publishes the routing).
-//   phase 2  work items (expert, 128-row panel of gate+up, K split), then
-//            (expert, 128-row panel of down, K half), dealt round-robin over
-//            the CTAs. One warp per CTA issues 1-D bulk copies of the items'
-//            packed tiles into a ring of shared-memory buffers; 16 warps
-//            decode the 2-bit codes in registers and multiply them with the
-//            tokens on the warp-level MMA (16 rows x 8 tokens x 16 columns,
-//            fp16 in, fp32 accumulate). Gate/up sums go to global memory; a
-//            per-expert counter releases that expert's down items, which form
-//            h = silu(g) * u and add w * W_down h into y with fp32 atomics.
-//
-// Why the warp MMA and not fp32 FMA: on this GPU, fp32 FMA dot products with
-// register dequantisation peak at about 2.2 TB/s of weight bytes for one
-// token and 1.0 TB/s for four (issue-bound: the multiply-adds per weight grow
-// with the tokens); the MMA takes the multiply-adds off the issue slots so
-// the stream can run at HBM speed for every token count up to 16. The
-// weights never touch shared memory after the copy: the codes are decoded
-// straight into MMA fragment registers.
+//            identically, each token's softmax top-k (one warp per token,
+//            warp max reductions, ties to the lower expert index), the
+//            renormalised weights and the per-expert token lists (bit masks
+//            of tokens, popcount ranks). CTA 0 publishes the routing.
+//   phase 2  work units (active expert e, 64-row slice p of its hidden
+//            layer), dealt round-robin over the CTAs. A unit needs no other
+//            unit: it streams the slice's gate and up rows over all of K
+//            (contiguous in the blob), forms h = silu(g) * u for the slice in
+//            shared memory, then streams the down columns the slice feeds
+//            (contiguous too) and adds w * W_down[:, slice] h into y with
+//            fp32 atomics. One warp per CTA issues 1-D bulk copies of 20 KB
+//            chunks into a ring of shared-memory buffers; 16 warps decode
+//            the 2-bit codes in registers straight into MMA fragments and
+//            multiply on the warp-level MMA (16 rows x 8 tokens x 16
+//            columns, fp16 in, fp32 accumulate).
 //
 // Exactness of the decode: a code c at mantissa bit p of an fp16 whose
 // exponent gives that bit the place value 1 is the exact value base_p + c
@@ -42,16 +39,27 @@
 // fp32 rounding. x (bf16) is exact in fp16 for |x| in [6.1e-5, 65504]; h is
 // rounded to fp16 (relative error <= 2^-11).
 //
-// Every wait (grid barrier, expert counter, copy barrier) is time-bounded;
-// on expiry the kernel records a timeout in the status word and unwinds.
+// Every wait (grid barrier, copy barrier) is time-bounded; on expiry the
+// kernel records a timeout in the status word and unwinds. Decisions to stop
+// are taken at barriers that OR a flag over all compute warps, so no warp is
+// left waiting at a barrier that the others skipped.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace strata {
 
-constexpr int kFusedComputeWarps = 16;                        // 8 row groups x 2
-constexpr int kFusedThreads = (kFusedComputeWarps + 1) * 32;  // + one copy-issue warp
-constexpr int kFusedMaxBuf = 8;
+constexpr int kFusedComputeWarps = 16;
+// 16 compute warps + one warp that issues the bulk copies (an issuing thread
+// can stall while the copy engine's queue is full, so no compute warp does).
+constexpr int kFusedThreads = (kFusedComputeWarps + 1) * 32;
+constexpr int kFusedMaxBuf = 16;
+constexpr int kGuSlicesPerChunk = 8;      // gate/up chunk: 8 K-slices x (gate, up) tiles = 20 KB
+constexpr int kDownPanelsPerChunk = 16;   // down chunk: 16 tiles of 64 d-rows = 20 KB
+constexpr uint32_t kChunkBytes = 20480;
+constexpr int kHStride = 64 + 8;          // fp16 row stride of h (halves)
+constexpr int kRouterRowsMax = 16;        // router rows per CTA (E <= 16 * number of CTAs)
 
 struct FusedArgs {
     const void *x;        // bf16 [T x d]; fp32 residual [T x d] when rms
@@ -64,36 +72,44 @@ struct FusedArgs {
     int rms;
     float eps;
     size_t ebytes, down_off;
-    int KS;               // gate/up K splits
+    ExpertStrides xs;
     int nbuf;
-    uint32_t buf_bytes;
     Workspace ws;
 };
 
-// fp16 row strides (halves): +8 makes consecutive token rows start 4 banks
-// apart, so the 8 rows x 4 column pairs of one B fragment load hit 32 banks
+// fp16 row stride of x (halves): +8 makes consecutive token rows start 4
+// banks apart, so the 8 rows x 4 column pairs of one B fragment load hit 32
+// different banks
 __host__ __device__ inline int hstride(int n) { return n + 8; }
 
 // shared-memory plan, identical on host and device
 struct FusedSmem {
-    size_t xh, xz, hh, hz, cand, sel_idx, sel_val, sel_w, cnt, off, act, ptok, pslot, pw, scan, bufs, total;
+    size_t xh, xz, red, hh, hz, lsm, sbias, sel_idx, sel_val, sel_w, mask, cnt, off, act, ptok, pslot, pw, scan, bufs, total;
 };
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~(size_t)15; }
 
-__host__ __device__ inline FusedSmem fused_plan(int T, int TT, int d, int f, int E, int k, int nbuf,
-                                               uint32_t buf_bytes) {
-    const int NS = TT <= 8 ? 8 : 16;  // token slots of the MMA n-tiles
+__host__ __device__ inline int token_slots(int TT) { return TT <= 8 ? 8 : 16; }
+// gate/up work split: KSPLIT groups of K slices x (16 / KSPLIT) groups of the
+// 8 (matrix, 16-row group) pairs of a 64-row slice; a warp loads a slice's
+// token fragments once for all its row groups
+__host__ __device__ inline constexpr int gu_ksplit(int TT) { return TT <= 8 ? 8 : 4; }
+
+__host__ __device__ inline FusedSmem fused_plan(int T, int TT, int d, int E, int k, int nbuf) {
+    const int NS = token_slots(TT);
     FusedSmem p;
     size_t o = 0;
     p.xh = o;      o = al16(o + (size_t)(T + 1) * hstride(d) * 2);   // + a zero row
     p.xz = o;      o = al16(o + (size_t)(T + 1) * (d / 32) * 4);
-    p.hh = o;      o = al16(o + (size_t)NS * hstride(f / 2) * 2);
-    p.hz = o;      o = al16(o + (size_t)NS * (f / 64) * 4);
-    p.cand = o;    o = al16(o + (size_t)kFusedComputeWarps * k * 8);
+    p.red = o;     o = al16(o + (size_t)gu_ksplit(TT) * 2 * 64 * TT * 4);  // [K group][gate/up][row][slot < TT]
+    p.hh = o;      o = al16(o + (size_t)NS * kHStride * 2);
+    p.hz = o;      o = al16(o + (size_t)NS * 2 * 4);
+    p.lsm = o;     o = al16(o + (size_t)T * kRouterRowsMax * 4 * 4);   // router partials [T][row][K quarter]
+    p.sbias = o;   o = al16(o + (size_t)kRouterRowsMax * 4);
     p.sel_idx = o; o = al16(o + (size_t)T * k * 4);
     p.sel_val = o; o = al16(o + (size_t)T * k * 4);
     p.sel_w = o;   o = al16(o + (size_t)T * k * 4);
+    p.mask = o;    o = al16(o + (size_t)E * 4);
     p.cnt = o;     o = al16(o + (size_t)E * 4);
     p.off = o;     o = al16(o + (size_t)(E + 1) * 4);
     p.act = o;     o = al16(o + (size_t)E * 4);
@@ -102,15 +118,19 @@ __host__ __device__ inline FusedSmem fused_plan(int T, int TT, int d, int f, int
     p.pw = o;      o = al16(o + (size_t)T * k * 4);
     p.scan = o;    o = al16(o + 64 * 4);
     o = (o + 127) & ~(size_t)127;
-    p.bufs = o;    o += (size_t)nbuf * buf_bytes;
+    p.bufs = o;    o += (size_t)nbuf * kChunkBytes;
     p.total = o;
     return p;
 }
 
-// monotone map of a float to uint32 (+0 and -0 both map to 0x80000000)
+// monotone map of a float to uint32 (+0 and -0 both map to 0x80000000);
+// every finite or infinite value maps above 0, the "taken" marker
 STRATA_DEV uint32_t ordered_key(float v) {
     uint32_t u = __float_as_uint(v + 0.0f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+STRATA_DEV float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // time-bounded spin until *ctr >= target (acquire); false on timeout/abort
@@ -136,8 +156,7 @@ STRATA_DEV bool wait_counter(const uint32_t *ctr, uint32_t target, uint32_t *sta
 STRATA_DEV void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFusedComputeWarps * 32) : "memory"); }
 
 // Barrier of the compute warps that also ORs a flag over them, so that every
-// compute thread takes the same decision (an abort seen by some threads
-// only would strand the others at the next barrier).
+// compute thread takes the same decision.
 STRATA_DEV bool compute_sync_any(bool v) {
     uint32_t r;
     asm volatile(
@@ -164,20 +183,33 @@ __host__ __device__ constexpr uint32_t step_magic(int j) {
 }
 __host__ __device__ constexpr float step_base(int j) { return j == 0 ? 16.f : j == 1 ? 64.f : j == 2 ? 256.f : 1024.f; }
 
-// One 16-row group x one 64-column tile x NT n-tiles of 8 token slots.
-//   wg, wg8  : this lane's code word (word t = lane & 3) of rows g and g+8
-//   sg, sg8  : the two fp16 block scales of rows g and g+8
-//   xb[n]    : fp16 input row of token slot (n*8 + lane/4), at the tile's column 0
-//   z0/z1[n] : per-block constants of token slots n*8 + 2t and n*8 + 2t + 1
-// out[n][0..3] += (rows g, g+8) x (slots 2t, 2t+1) dot products.
-template <int NT>
-STRATA_DEV void tile_mma(uint32_t wg, uint32_t wg8, uint32_t sg, uint32_t sg8, const __half *const (&xb)[NT],
-                         const float *const (&z0)[NT], const float *const (&z1)[NT], int nt_active,
-                         float (&out)[NT][4]) {
+// The A-side words of one 16-row group of a tile: lane (g, t) reads word t
+// of rows g and g+8 and the two rows' block scales.
+struct TileRows {
+    uint32_t wg, wg8, sg, sg8;
+};
+STRATA_DEV TileRows load_rows(const uint8_t *tile, int gr) {
     const int t = threadIdx.x & 3;
-    const uint32_t v8g = wg >> 8, v8g8 = wg8 >> 8;
-    const float2 s_g = __half22float2(*reinterpret_cast<const __half2 *>(&sg));
-    const float2 s_g8 = __half22float2(*reinterpret_cast<const __half2 *>(&sg8));
+    TileRows r;
+    r.wg = *reinterpret_cast<const uint32_t *>(tile + 16 * gr + 4 * t);
+    r.wg8 = *reinterpret_cast<const uint32_t *>(tile + 16 * (gr + 8) + 4 * t);
+    r.sg = *reinterpret_cast<const uint32_t *>(tile + kTileScaleOffset + 4 * gr);
+    r.sg8 = *reinterpret_cast<const uint32_t *>(tile + kTileScaleOffset + 4 * (gr + 8));
+    return r;
+}
+
+// One 16-row group x one 64-column tile x NT n-tiles of 8 token slots.
+// B fragments and block constants come from `bsrc(n, j, b0, b1)` and
+// `zsrc(n, blk, z_a, z_b)` (token slots n*8 + 2t and n*8 + 2t + 1).
+// out[n][0..3] += (rows g, g+8) x (slots 2t, 2t+1) dot products; with
+// ODD false (one token: only slot 0 is real) the odd slots are left alone.
+// NT is the number of n-tiles that hold tokens: no per-tile predicate sits
+// between the MMAs (it costs about half the loop's throughput).
+template <int NT, bool ODD, typename BSrc, typename ZSrc>
+STRATA_DEV void tile_mma(const TileRows &w, BSrc bsrc, ZSrc zsrc, float (&out)[NT][4]) {
+    const uint32_t v8g = w.wg >> 8, v8g8 = w.wg8 >> 8;
+    const float2 s_g = __half22float2(*reinterpret_cast<const __half2 *>(&w.sg));
+    const float2 s_g8 = __half22float2(*reinterpret_cast<const __half2 *>(&w.sg8));
 #pragma unroll
     for (int blk = 0; blk < 2; ++blk) {
         float acc[NT][4];
@@ -189,55 +221,125 @@ STRATA_DEV void tile_mma(uint32_t wg, uint32_t wg8, uint32_t sg, uint32_t sg8, c
         for (int jj = 0; jj < 2; ++jj) {
             const int j = 2 * blk + jj;
             const uint32_t m = 0x00030003u << (6 - 2 * j), g = step_magic(j);
-            const uint32_t a[4] = {(wg & m) | g, (wg8 & m) | g, (v8g & m) | g, (v8g8 & m) | g};
+            const uint32_t a[4] = {(w.wg & m) | g, (w.wg8 & m) | g, (v8g & m) | g, (v8g8 & m) | g};
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                if (n < nt_active) {
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t *>(xb[n] + 16 * j + 2 * t);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t *>(xb[n] + 16 * j + 8 + 2 * t);
-                    mma16816(acc[n], a, b0, b1);
-                }
+                uint32_t b0, b1;
+                bsrc(n, j, b0, b1);
+                mma16816(acc[n], a, b0, b1);
             }
         }
         const float sb = blk ? s_g.y : s_g.x, sb8 = blk ? s_g8.y : s_g8.x;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            if (n < nt_active) {
-                const float za = z0[n][blk], zb = z1[n][blk];
-                out[n][0] = fmaf(sb, acc[n][0] - za, out[n][0]);
+            float za, zb;
+            zsrc(n, blk, za, zb);
+            out[n][0] = fmaf(sb, acc[n][0] - za, out[n][0]);
+            out[n][2] = fmaf(sb8, acc[n][2] - za, out[n][2]);
+            if (ODD) {
                 out[n][1] = fmaf(sb, acc[n][1] - zb, out[n][1]);
-                out[n][2] = fmaf(sb8, acc[n][2] - za, out[n][2]);
                 out[n][3] = fmaf(sb8, acc[n][3] - zb, out[n][3]);
             }
         }
     }
 }
 
-// Per-block constant of one staged fp16 row (columns in 64-column tiles):
-// z[b] = sum_{16-col steps j of block b} base_j * X_j + 1.5 * X_b.
-STRATA_DEV float block_constant(const __half *row, int b) {
-    const int j0 = 2 * (b & 1);
-    float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        x0 += __half2float(row[32 * b + c]);
-        x1 += __half2float(row[32 * b + 16 + c]);
+// Per-block constants of one staged fp16 row (columns in 64-column tiles),
+// one warp: z[b] = sum over the block's columns k of (base_j(k) + 1.5) x_k,
+// i.e. sum_j base_j X_j + 1.5 X_b. Lane l reads columns 2l, 2l+1 of each
+// tile (step j = l / 8, block l / 16) and the 16 lanes of a block reduce by
+// shuffles, so the reads are conflict-free.
+STRATA_DEV void row_block_constants(const __half *row, int ncols, float *z) {
+    const int lane = threadIdx.x & 31;
+    const float wgt = step_base(lane >> 3) + 1.5f;
+    for (int c0 = 0; c0 < ncols; c0 += 64) {
+        const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(row + c0 + 2 * lane));
+        float sum = wgt * (v.x + v.y);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 8);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        if ((lane & 15) == 0) z[c0 / 32 + (lane >> 4)] = sum;
     }
-    return step_base(j0) * x0 + step_base(j0 + 1) * x1 + 1.5f * (x0 + x1);
 }
 
-// ------------------------------------------------------------ top-k helpers
-// A lane's candidates: KPL (ordered logit, expert) pairs; 0 / 0x7fffffff mark
-// an empty slot. `better` orders by logit descending, then index ascending.
-STRATA_DEV bool better(uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) { return ka > kb || (ka == kb && ia < ib); }
+// One gate/up K slice for the warp's RGM (matrix, row group) pairs: the
+// slice's token fragments are loaded once and reused for every pair.
+template <int NTA, int NT, int RGM, bool ODD>
+STRATA_DEV void gu_slice(const uint8_t *tiles, const __half *const (&xb)[NT], const float *const (&z0)[NT],
+                         const float *const (&z1)[NT], int col0, int rgm0, int g, float (&out)[RGM][NT][4]) {
+    uint32_t bf[NTA][4][2];
+    float2 zA[NTA], zB[NTA];
+#pragma unroll
+    for (int n = 0; n < NTA; ++n) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            bf[n][j][0] = *reinterpret_cast<const uint32_t *>(xb[n] + col0 + 16 * j);
+            bf[n][j][1] = *reinterpret_cast<const uint32_t *>(xb[n] + col0 + 16 * j + 8);
+        }
+        zA[n] = *reinterpret_cast<const float2 *>(z0[n] + col0 / 32);
+        zB[n] = ODD ? *reinterpret_cast<const float2 *>(z1[n] + col0 / 32) : zA[n];
+    }
+#pragma unroll
+    for (int r = 0; r < RGM; ++r) {
+        const int rgm = rgm0 + r, m = rgm >> 2, gr = 16 * (rgm & 3) + g;
+        const TileRows w = load_rows(tiles + m * kTileBytes, gr);
+        tile_mma<NTA, ODD>(
+            w,
+            [&](int n, int j, uint32_t &b0, uint32_t &b1) {
+                b0 = bf[n][j][0];
+                b1 = bf[n][j][1];
+            },
+            [&](int n, int blk, float &za, float &zb) {
+                za = blk ? zA[n].y : zA[n].x;
+                zb = blk ? zB[n].y : zB[n].x;
+            },
+            reinterpret_cast<float(&)[NTA][4]>(out[r]));
+    }
+}
 
-// Local top-k of one warp: each lane sorts its KPL pairs (register bitonic
-// network), then k rounds of a warp max over the lanes' heads (REDUX max on
-// the key, REDUX min on the index among the lanes holding that key); the
-// winning lane pops its head. Writes k (key, expert) pairs, expert -1 when
-// the warp has fewer than k candidates.
+// One down tile row group with h fragments and block constants held in
+// registers for the whole unit.
+template <int NTA, int NT, bool ODD>
+STRATA_DEV void down_rows(const TileRows &w, const uint32_t (&bf)[NT][4][2], const float (&zf)[NT][2][2],
+                          float (&o)[NT][4]) {
+    tile_mma<NTA, ODD>(
+        w,
+        [&](int n, int j, uint32_t &b0, uint32_t &b1) {
+            b0 = bf[n][j][0];
+            b1 = bf[n][j][1];
+        },
+        [&](int n, int blk, float &za, float &zb) {
+            za = zf[n][blk][0];
+            zb = zf[n][blk][1];
+        },
+        reinterpret_cast<float(&)[NTA][4]>(o));
+}
+
+// ------------------------------------------------------------ top-k
+// One warp, one token. Lane l holds the logits of experts KPL*l ..
+// KPL*l + KPL - 1 as ordered keys, sorted in registers (bitonic network,
+// key descending, then expert ascending). Among equal keys the lowest lane
+// holds the lowest expert index, so each of the k rounds takes the warp max
+// of the lanes' heads and the lowest lane holding it (ballot), which pops
+// its head.
 template <int KPL>
-STRATA_DEV void warp_topk(uint32_t (&kk)[KPL], uint32_t (&id)[KPL], int k, uint32_t *ok, int *oid) {
+STRATA_DEV void token_topk(const float *logits, int t, int E, int k, int *sel_idx, float *sel_val) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[KPL];
+    int pos[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; i += 4) {
+        const int e = KPL * lane + i;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < E) v = __ldcg(reinterpret_cast<const float4 *>(logits + (size_t)t * E + e));  // E % 4 == 0
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            key[i + q] = e + q < E ? ordered_key(vv[q]) : 0u;  // 0: below every real key
+            pos[i + q] = i + q;
+        }
+    }
 #pragma unroll
     for (int size = 2; size <= KPL; size <<= 1)
 #pragma unroll
@@ -246,79 +348,60 @@ STRATA_DEV void warp_topk(uint32_t (&kk)[KPL], uint32_t (&id)[KPL], int k, uint3
             for (int i = 0; i < KPL; ++i) {
                 const int j = i ^ stride;
                 if (j > i) {
+                    // ascending blocks reversed: the network sorts descending by (key, -position)
                     const bool desc = (i & size) == 0;
-                    const bool sw = desc ? better(kk[j], id[j], kk[i], id[i]) : better(kk[i], id[i], kk[j], id[j]);
-                    const uint32_t tk = kk[i], ti = id[i];
-                    kk[i] = sw ? kk[j] : tk;
-                    id[i] = sw ? id[j] : ti;
-                    kk[j] = sw ? tk : kk[j];
-                    id[j] = sw ? ti : id[j];
+                    const bool jfirst = key[j] > key[i] || (key[j] == key[i] && pos[j] < pos[i]);
+                    const bool sw = desc ? jfirst : !jfirst;
+                    const uint32_t tk = key[i];
+                    const int tp = pos[i];
+                    key[i] = sw ? key[j] : tk;
+                    pos[i] = sw ? pos[j] : tp;
+                    key[j] = sw ? tk : key[j];
+                    pos[j] = sw ? tp : pos[j];
                 }
             }
-    const int lane = threadIdx.x & 31;
     for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(0xffffffffu, kk[0]);
-        const uint32_t w = __reduce_min_sync(0xffffffffu, (kk[0] == m) ? id[0] : 0x7fffffffu);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+        const int wl = __ffs(__ballot_sync(0xffffffffu, key[0] == m)) - 1;
+        const int wp = __shfl_sync(0xffffffffu, pos[0], wl);
         if (lane == 0) {
-            ok[j] = m;
-            oid[j] = m ? (int)w : -1;
+            sel_idx[j] = KPL * wl + wp;
+            sel_val[j] = key_value(m);
         }
-        if (m && id[0] == w) {
+        if (lane == wl) {
 #pragma unroll
             for (int i = 0; i + 1 < KPL; ++i) {
-                kk[i] = kk[i + 1];
-                id[i] = id[i + 1];
+                key[i] = key[i + 1];
+                pos[i] = pos[i + 1];
             }
-            kk[KPL - 1] = 0u;
-            id[KPL - 1] = 0x7fffffffu;
+            key[KPL - 1] = 0u;
         }
     }
-}
-
-template <int KPL>
-STRATA_DEV void chunk_topk(const float *lpart, const float *bias, int t, int E, int e0, int e1, int k, uint32_t *ok,
-                           int *oid) {
-    const int lane = threadIdx.x & 31;
-    uint32_t kk[KPL], id[KPL];
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-        kk[i] = 0u;
-        id[i] = 0x7fffffffu;
-        const int e = e0 + lane + 32 * i;
-        if (e < e1) {
-            const float4 pq = __ldcg(reinterpret_cast<const float4 *>(lpart + ((size_t)t * E + e) * 4));
-            float l = ((pq.x + pq.y) + pq.z) + pq.w;  // fixed order over the K quarters
-            if (bias) l += bias[e];
-            kk[i] = ordered_key(l);
-            id[i] = (uint32_t)e;
-        }
-    }
-    warp_topk<KPL>(kk, id, k, ok, oid);
 }
 
 template <int TT>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], wbar;
+    __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar;
     __shared__ int s_abort;
-    __shared__ float s_red[kFusedComputeWarps][2];
     constexpr int NT = TT <= 8 ? 1 : 2;  // MMA n-tiles of 8 token slots
+    constexpr int NS = NT * 8;
 
     const int T = a.T, d = a.d, f = a.f, E = a.E, k = a.k;
-    const int FH = f / 2, dpx = hstride(d), dph = hstride(FH);
+    const int dpx = hstride(d);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool producer = warp == kFusedComputeWarps;
     const int G = gridDim.x, b = blockIdx.x;
-    const FusedSmem sp = fused_plan(T, TT, d, f, E, k, a.nbuf, a.buf_bytes);
+    const FusedSmem sp = fused_plan(T, TT, d, E, k, a.nbuf);
     __half *xh = reinterpret_cast<__half *>(smem + sp.xh);
     float *xz = reinterpret_cast<float *>(smem + sp.xz);
+    float *red = reinterpret_cast<float *>(smem + sp.red);
     __half *hh = reinterpret_cast<__half *>(smem + sp.hh);
     float *hz = reinterpret_cast<float *>(smem + sp.hz);
-    uint32_t *cand_k = reinterpret_cast<uint32_t *>(smem + sp.cand);
-    int *cand_i = reinterpret_cast<int *>(smem + sp.cand) + kFusedComputeWarps * k;
     int *sel_idx = reinterpret_cast<int *>(smem + sp.sel_idx);
     float *sel_val = reinterpret_cast<float *>(smem + sp.sel_val);
     float *sel_w = reinterpret_cast<float *>(smem + sp.sel_w);
+    uint32_t *mask = reinterpret_cast<uint32_t *>(smem + sp.mask);
     int *cnt = reinterpret_cast<int *>(smem + sp.cnt);
     int *off = reinterpret_cast<int *>(smem + sp.off);
     int *act = reinterpret_cast<int *>(smem + sp.act);
@@ -327,49 +410,82 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     float *pw = reinterpret_cast<float *>(smem + sp.pw);
     int *scan = reinterpret_cast<int *>(smem + sp.scan);
     uint8_t *bufs = smem + sp.bufs;
-    float *lpart = a.ws.lpart;  // router partial sums [T][E][4]
-    uint32_t *sync = a.ws.sync;  // [0] grid barrier, [1] exit count, [2..2+E) per-expert gate/up counters
+    float *logits = a.ws.lpart;  // router logits [T][E] (+ bias)
+    float *lsm = reinterpret_cast<float *>(smem + sp.lsm);
+    float *sbias = reinterpret_cast<float *>(smem + sp.sbias);
+    uint32_t *sync = a.ws.sync;  // [0] grid barrier, [1] exit count
     uint32_t *status = a.ws.status;
 
     // ---------------------------------------------------------------- phase 0
     const int r0 = (int)((long long)E * b / G), r1 = (int)((long long)E * (b + 1) / G);
     const int nr = r1 - r0;
+    const uint32_t xbytes = (uint32_t)T * d * 2;
+    const uint32_t xoff = (xbytes + 127) & ~127u;
     const uint32_t wbytes = (uint32_t)nr * d * 4;
-    const bool wstaged = nr > 0 && wbytes <= (uint32_t)a.nbuf * a.buf_bytes;
-    if (producer && lane == 0) {
+    const uint32_t ring = (uint32_t)a.nbuf * kChunkBytes;
+    const bool xstaged = !a.rms && xbytes <= ring;
+    const uint32_t woff = xstaged ? xoff : 0u;
+    const bool wstaged = nr > 0 && woff + wbytes <= ring;
+    if (warp == kFusedComputeWarps && lane == 0) {
         for (int i = 0; i < a.nbuf; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kFusedComputeWarps);
         }
+        mbar_init(&xbar, 1);
         mbar_init(&wbar, 1);
         s_abort = 0;
         fence_mbar_init();
+        if (xstaged) {
+            mbar_arrive_expect_tx(&xbar, xbytes);
+            bulk_g2s(bufs, a.x, xbytes, &xbar);
+        }
         if (wstaged) {  // this CTA's router rows, one bulk copy
             mbar_arrive_expect_tx(&wbar, wbytes);
-            bulk_g2s(bufs, a.W + (size_t)r0 * d, wbytes, &wbar);
+            bulk_g2s(bufs + woff, a.W + (size_t)r0 * d, wbytes, &wbar);
         }
+    }
+    if (tid < nr) {  // the router bias of this CTA's rows, without waiting for it here
+        if (a.bias)
+            cp_async4(sbias + tid, a.bias + r0 + tid);
+        else
+            sbias[tid] = 0.f;
     }
     __syncthreads();
     if (!producer) {
-        if (a.rms) {  // stack glue: bf16(RMSNorm(x)) of the fp32 residual
-            for (int t = 0; t < T; ++t) {
-                const float *xr = static_cast<const float *>(a.x) + (size_t)t * d;
+        if (!a.accumulate && !a.rms) {  // zero this CTA's slice of y
+            const size_t n = (size_t)T * d, lo = n * b / G, hi = n * (b + 1) / G;
+            for (size_t i = lo + tid; i < hi; i += 512) a.y[i] = 0.f;
+        }
+        if (a.rms) {  // stack glue: bf16(RMSNorm) of the fp32 residual, one warp per token
+            for (int t = warp; t < T; t += kFusedComputeWarps) {
+                const float4 *xr = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (size_t)t * d);
                 float ss = 0.f;
-                for (int c = tid; c < d; c += 512) ss = fmaf(xr[c], xr[c], ss);
+                for (int c = lane; c < d / 4; c += 32) {
+                    const float4 v = xr[c];
+                    ss = fmaf(v.x, v.x, ss);
+                    ss = fmaf(v.y, v.y, ss);
+                    ss = fmaf(v.z, v.z, ss);
+                    ss = fmaf(v.w, v.w, ss);
+                }
                 ss = warp_sum(ss);
-                if (lane == 0) s_red[warp][t & 1] = ss;
-                compute_sync();
-                float tot = 0.f;
-#pragma unroll
-                for (int w2 = 0; w2 < kFusedComputeWarps; ++w2) tot += s_red[w2][t & 1];
-                const float inv = 1.0f / sqrtf(tot / (float)d + a.eps);
-                for (int c = tid; c < d; c += 512)
-                    xh[(size_t)t * dpx + c] = __float2half_rn(__bfloat162float(__float2bfloat16_rn(xr[c] * inv)));
+                const float inv = 1.0f / sqrtf(ss / (float)d + a.eps);
+                for (int c = lane; c < d / 4; c += 32) {
+                    const float4 v = xr[c];
+                    __half2 *dst = reinterpret_cast<__half2 *>(xh + (size_t)t * dpx + 4 * c);
+                    dst[0] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.x * inv)),
+                                               __bfloat162float(__float2bfloat16_rn(v.y * inv)));
+                    dst[1] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.z * inv)),
+                                               __bfloat162float(__float2bfloat16_rn(v.w * inv)));
+                }
             }
         } else {
             const uint4 *xv = static_cast<const uint4 *>(a.x);
+            if (xstaged) {
+                mbar_wait(&xbar, 0, status, &s_abort);
+                xv = reinterpret_cast<const uint4 *>(bufs);
+            }
             for (int i = tid; i < T * d / 8; i += 512) {
-                const uint4 v = __ldg(xv + i);
+                const uint4 v = xv[i];
                 const int t = (i * 8) / d, c = (i * 8) % d;
                 const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t h4[4];
@@ -382,43 +498,56 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 *reinterpret_cast<uint4 *>(xh + (size_t)t * dpx + c) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
             }
         }
-        for (int c = tid; c < d; c += 512) xh[(size_t)T * dpx + c] = __float2half_rn(0.f);  // zero row
-        if (!a.accumulate && !a.rms) {  // zero this CTA's slice of y
-            const size_t n = (size_t)T * d, lo = n * b / G, hi = n * (b + 1) / G;
-            for (size_t i = lo + tid; i < hi; i += 512) a.y[i] = 0.f;
-        }
+        for (int c = tid; c < d / 2; c += 512)  // zero row (empty MMA token slots)
+            reinterpret_cast<uint32_t *>(xh + (size_t)T * dpx)[c] = 0u;
         compute_sync();
-        for (int i = tid; i < (T + 1) * (d / 32); i += 512)  // per-block constants of x
-            xz[i] = block_constant(xh + (size_t)(i / (d / 32)) * dpx, i % (d / 32));
+        for (int r = warp; r <= T; r += kFusedComputeWarps)  // per-block constants of x (and the zero row)
+            row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
+        // router: warp -> (row, quarter of K); each lane keeps 16 K-values of
+        // W in registers per 512-column step and walks the tokens
         if (wstaged) mbar_wait(&wbar, 0, status, &s_abort);
-        const int q4 = d / 4;  // router: warp -> (row, quarter of K), partial sums
+        const int q4 = d / 4;
         for (int u = warp; u < nr * 4 && !s_abort; u += kFusedComputeWarps) {
             const int rr = u / 4, kq = u % 4;
-            const float4 *w4 = wstaged ? reinterpret_cast<const float4 *>(bufs + ((size_t)rr * d + (size_t)kq * q4) * 4)
-                                       : reinterpret_cast<const float4 *>(a.W + (size_t)(r0 + rr) * d + (size_t)kq * q4);
-            float acc[TT];
+            const float *wrow = wstaged ? reinterpret_cast<const float *>(bufs + woff) + (size_t)rr * d
+                                        : a.W + (size_t)(r0 + rr) * d;
+            const int cbase = kq * q4;
+            for (int c0 = 0; c0 < q4; c0 += 512) {
+                const int ncol = min(512, q4 - c0);  // a multiple of 32 (d is a multiple of 128)
+                float4 wv[4];
 #pragma unroll
-            for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-            for (int i = lane; i < q4 / 4; i += 32) {
-                const float4 wv = w4[i];
-                const int c = kq * q4 + 4 * i;
+                for (int i = 0; i < 4; ++i)
+                    wv[i] = 128 * i + 4 * lane < ncol
+                                ? *reinterpret_cast<const float4 *>(wrow + cbase + c0 + 128 * i + 4 * lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int t = 0; t < T; ++t) {
+                    const __half *xr = xh + (size_t)t * dpx + cbase + c0;
+                    float acc = 0.f;
 #pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    if (t < T) {
-                        const __half2 *xp = reinterpret_cast<const __half2 *>(xh + (size_t)t * dpx + c);
-                        const float2 x01 = __half22float2(xp[0]), x23 = __half22float2(xp[1]);
-                        acc[t] = fmaf(wv.x, x01.x, acc[t]);
-                        acc[t] = fmaf(wv.y, x01.y, acc[t]);
-                        acc[t] = fmaf(wv.z, x23.x, acc[t]);
-                        acc[t] = fmaf(wv.w, x23.y, acc[t]);
+                    for (int i = 0; i < 4; ++i) {
+                        if (128 * i + 4 * lane < ncol) {
+                            const __half2 *xp = reinterpret_cast<const __half2 *>(xr + 128 * i + 4 * lane);
+                            const float2 x01 = __half22float2(xp[0]), x23 = __half22float2(xp[1]);
+                            acc = fmaf(wv[i].x, x01.x, acc);
+                            acc = fmaf(wv[i].y, x01.y, acc);
+                            acc = fmaf(wv[i].z, x23.x, acc);
+                            acc = fmaf(wv[i].w, x23.y, acc);
+                        }
+                    }
+                    acc = warp_sum(acc);
+                    if (lane == 0) {
+                        float *dst = lsm + ((size_t)t * kRouterRowsMax + rr) * 4 + kq;
+                        *dst = (c0 == 0) ? acc : *dst + acc;
                     }
                 }
             }
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const float v = warp_sum(acc[t]);
-                if (lane == 0 && t < T) lpart[((size_t)t * E + r0 + rr) * 4 + kq] = v;
-            }
+        }
+        if (tid < nr) cp_async_wait_all();
+        compute_sync();
+        for (int i = tid; i < T * nr; i += 512) {  // logits: the K quarters in a fixed order, + bias
+            const int t = i / nr, rr = i % nr;
+            const float *pq = lsm + ((size_t)t * kRouterRowsMax + rr) * 4;
+            logits[(size_t)t * E + r0 + rr] = (((pq[0] + pq[1]) + pq[2]) + pq[3]) + sbias[rr];
         }
     }
     __syncthreads();
@@ -431,54 +560,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
 
     // ---------------------------------------------------------------- phase 1
     if (!s_abort && !producer) {
-        const int wpt = T <= 4 ? 4 : T <= 8 ? 2 : 1;  // warps per token
-        const int chunk = (E + wpt - 1) / wpt;
-        const int need = (chunk + 31) / 32;  // candidates per lane
-        for (int u = warp; u < T * wpt; u += kFusedComputeWarps) {
-            const int t = u / wpt, part = u % wpt;
-            const int e0 = part * chunk, e1 = min(E, e0 + chunk);
-            uint32_t *ok = cand_k + (size_t)u * k;
-            int *oi = cand_i + (size_t)u * k;
-            if (TT < 16) {
-                if (need <= 4) chunk_topk<4>(lpart, a.bias, t, E, e0, e1, k, ok, oi);
-                else chunk_topk<8>(lpart, a.bias, t, E, e0, e1, k, ok, oi);
-            } else {
-                if (need <= 8) chunk_topk<8>(lpart, a.bias, t, E, e0, e1, k, ok, oi);
-                else if (need <= 16) chunk_topk<16>(lpart, a.bias, t, E, e0, e1, k, ok, oi);
-                else chunk_topk<32>(lpart, a.bias, t, E, e0, e1, k, ok, oi);
-            }
+        for (int e = tid; e < E; e += 512) mask[e] = 0u;
+        if (warp < T) {  // one warp per token
+            token_topk<16>(logits, warp, E, k, sel_idx + warp * k, sel_val + warp * k);
+            __syncwarp();
+            // renormalised softmax weights over the k selected
+            const float vmax = sel_val[warp * k];
+            float ex = 0.f;
+            for (int j = lane; j < k; j += 32) ex += expf(sel_val[warp * k + j] - vmax);
+            const float den = warp_sum(ex);
+            for (int j = lane; j < k; j += 32) sel_w[warp * k + j] = expf(sel_val[warp * k + j] - vmax) / den;
         }
         compute_sync();
-        const int nc = wpt * k;  // merge: rank of each candidate among its token's candidates
-        for (int c = tid; c < T * nc; c += 512) {
-            const int t = c / nc;
-            if (cand_i[c] < 0) continue;
-            const uint32_t kc = cand_k[c], ic = (uint32_t)cand_i[c];
-            int rank = 0;
-            for (int c2 = t * nc; c2 < (t + 1) * nc; ++c2)
-                rank += cand_i[c2] >= 0 && better(cand_k[c2], (uint32_t)cand_i[c2], kc, ic);
-            if (rank < k) {
-                sel_idx[t * k + rank] = (int)ic;
-                sel_val[t * k + rank] = __uint_as_float((kc & 0x80000000u) ? (kc & 0x7FFFFFFFu) : ~kc);
-            }
-        }
+        for (int i = tid; i < T * k; i += 512) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
         compute_sync();
-        for (int i = tid; i < T * k; i += 512) {  // renormalised softmax weights
-            const int t = i / k;
-            const float vmax = sel_val[t * k];
-            float den = 0.f;
-            for (int j = 0; j < k; ++j) den += expf(sel_val[t * k + j] - vmax);
-            sel_w[i] = expf(sel_val[i] - vmax) / den;
-        }
-        for (int e = tid; e < E; e += 512) {  // per-expert counts
-            int c = 0;
-            for (int i = 0; i < T * k; ++i) c += (sel_idx[i] == e);
-            cnt[e] = c;
-        }
-        compute_sync();
-        {  // exclusive scans of the counts and of (count > 0), 2 experts per thread
+        {  // counts and exclusive scans of the counts and of (count > 0), 2 experts per thread
             const int e0 = 2 * tid;
-            const int c0 = e0 < E ? cnt[e0] : 0, c1 = e0 + 1 < E ? cnt[e0 + 1] : 0;
+            const int c0 = e0 < E ? __popc(mask[e0]) : 0, c1 = e0 + 1 < E ? __popc(mask[e0 + 1]) : 0;
             const int a0 = c0 > 0, a1 = c1 > 0;
             int sc = c0 + c1, sa = a0 + a1;
 #pragma unroll
@@ -514,10 +612,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             const int bc = warp ? scan[warp - 1] : 0, ba = warp ? scan[32 + warp - 1] : 0;
             const int ic = bc + sc - (c0 + c1), ia = ba + sa - (a0 + a1);
             if (e0 < E) {
+                cnt[e0] = c0;
                 off[e0] = ic;
                 if (a0) act[ia] = e0;
             }
             if (e0 + 1 < E) {
+                cnt[e0 + 1] = c1;
                 off[e0 + 1] = ic + c0;
                 if (a1) act[ia + a0] = e0 + 1;
             }
@@ -526,9 +626,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         compute_sync();
         for (int p = tid; p < T * k; p += 512) {  // pairs in (expert, ascending token) order
             const int t = p / k, j = p % k, e = sel_idx[p];
-            int rank = 0;
-            for (int i = 0; i < t * k; ++i) rank += (sel_idx[i] == e);
-            const int pos = off[e] + rank;
+            const int pos = off[e] + __popc(mask[e] & ((1u << t) - 1u));
             ptok[pos] = t;
             pslot[pos] = j;
             pw[pos] = sel_w[p];
@@ -555,198 +653,232 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     const int n_act = s_abort ? 0 : scan[32 + kFusedComputeWarps - 1];
 
     // ---------------------------------------------------------------- phase 2
-    const int KS = a.KS, SL = (d / 64) / KS;
-    const int P1 = f / 128, P2 = d / 128, SLD = FH / 64;
-    const int n_gu = n_act * P1 * KS, n_dn = n_act * P2 * 2, n_all = n_gu + n_dn;
-    const int nq = (n_all > b) ? (n_all - b + G - 1) / G : 0;
-    const int NPD = kDecMaxT * k;
+    const int FP = f / 64;   // 64-row slices of the hidden layer
+    const int SLK = d / 64;  // K slices of gate/up = 64-row panels of down
+    const int nG = (SLK + kGuSlicesPerChunk - 1) / kGuSlicesPerChunk;
+    const int nD = (SLK + kDownPanelsPerChunk - 1) / kDownPanelsPerChunk;
+    const int n_units = n_act * FP;
+    const int nq = (n_units > b) ? (n_units - b + G - 1) / G : 0;
+    // chunk i of unit u: its source and size
+    auto chunk_src = [&](int u, int i, uint32_t &bytes) -> const uint8_t * {
+        const uint8_t *ebase = a.blob + (size_t)act[u / FP] * a.ebytes;
+        const int p = u % FP;
+        if (i < nG) {
+            const int s0 = i * kGuSlicesPerChunk, ns = min(kGuSlicesPerChunk, SLK - s0);
+            bytes = (uint32_t)ns * 2u * kTileBytes;
+            return ebase + (size_t)p * a.xs.gu_panel + (size_t)s0 * a.xs.gu_slice;
+        }
+        const int p0 = (i - nG) * kDownPanelsPerChunk, np = min(kDownPanelsPerChunk, SLK - p0);
+        bytes = (uint32_t)np * kTileBytes;
+        return ebase + a.down_off + (size_t)p * a.xs.dn_slice + (size_t)p0 * a.xs.dn_panel;
+    };
 
+    const int per = nG + nD, total = nq * per;
     if (producer) {
         // ------------------------------------------------ copy issue (one lane)
-        if (lane == 0) {
-            int q = 0;
-            for (; q < nq && !s_abort; ++q) {
-                const int it = b + q * G, bi = q % a.nbuf;
-                if (q >= a.nbuf && !mbar_wait(&empty[bi], (uint32_t)(((q / a.nbuf) - 1) & 1), status, &s_abort))
+        if (warp == kFusedComputeWarps && lane == 0) {
+            fence_proxy_async_smem();  // the staging reads of the ring (phase 0) come before these writes
+            int c = 0;
+            bool ok = !s_abort;
+            for (; c < total && ok; ++c) {
+                const int bi = c % a.nbuf;
+                if (c >= a.nbuf && !mbar_wait(&empty[bi], (uint32_t)(((c / a.nbuf) - 1) & 1), status, &s_abort)) {
+                    ok = false;
                     break;
-                const uint8_t *src;
-                uint32_t bytes;
-                if (it < n_gu) {
-                    const int u = it / (P1 * KS), r = it % (P1 * KS), p = r / KS, ks = r % KS;
-                    src = a.blob + (size_t)act[u] * a.ebytes + ((size_t)p * (d / 64) + (size_t)ks * SL) * 5120;
-                    bytes = (uint32_t)SL * 5120u;
-                } else {
-                    const int i2 = it - n_gu;
-                    const int u = i2 / (P2 * 2), r = i2 % (P2 * 2), p = r / 2, kd = r % 2;
-                    src = a.blob + (size_t)act[u] * a.ebytes + a.down_off +
-                          ((size_t)p * (f / 64) + (size_t)kd * SLD) * 2560;
-                    bytes = (uint32_t)SLD * 2560u;
                 }
+                uint32_t bytes;
+                const uint8_t *src = chunk_src(b + (c / per) * G, c % per, bytes);
                 mbar_arrive_expect_tx(&full[bi], bytes);
-                bulk_g2s(bufs + (size_t)bi * a.buf_bytes, src, bytes, &full[bi]);
+                bulk_g2s(bufs + (size_t)bi * kChunkBytes, src, bytes, &full[bi]);
+                if (c == a.nbuf - 1 || c == total - 1) {
+                    // Every CTA, the idle ones too, asks L2 for a share of the
+                    // chunks that their owners copy only after their first
+                    // ring's worth, so that those copies find their data in L2.
+                    for (int ci = b; ci < n_units * per; ci += G) {
+                        const int u = ci / per, j = (u / G) * per + ci % per;  // position in the owner's sequence
+                        if (j < a.nbuf) continue;
+                        uint32_t pb;
+                        const uint8_t *ps = chunk_src(u, ci % per, pb);
+                        prefetch_l2(ps, pb);
+                    }
+                }
             }
+            if (total == 0)
+                for (int ci = b; ci < n_units * per; ci += G) {
+                    const int u = ci / per, j = (u / G) * per + ci % per;
+                    if (j < a.nbuf) continue;
+                    uint32_t pb;
+                    const uint8_t *ps = chunk_src(u, ci % per, pb);
+                    prefetch_l2(ps, pb);
+                }
             // copies still in flight (only after an abort) land before exit
-            for (int j = (q > a.nbuf ? q - a.nbuf : 0); j < q; ++j)
+            for (int j = (c > a.nbuf ? c - a.nbuf : 0); j < c; ++j)
                 mbar_wait(&full[j % a.nbuf], (uint32_t)((j / a.nbuf) & 1), status, nullptr);
+            if (xstaged && s_abort) mbar_wait(&xbar, 0, status, nullptr);
             if (wstaged && s_abort) mbar_wait(&wbar, 0, status, nullptr);
         }
     } else {
         // ------------------------------------------------ compute warps
+        constexpr int KSPLIT = gu_ksplit(TT);
+        constexpr int RGM = 8 / (kFusedComputeWarps / KSPLIT);  // (matrix, row group) pairs per warp
+        constexpr bool ODD = TT > 1;
         const int t4 = lane & 3, g = lane >> 2;
-        const int rg = warp & 7;  // 16-row group of the 128-row panel
+        const int kq = warp % KSPLIT;            // gate/up: K-slice group
+        const int rgm0 = (warp / KSPLIT) * RGM;  // gate/up: first (matrix, row group) pair
+        int c = 0;
+        bool bad = false, stop = false;
         for (int q = 0; q < nq; ++q) {
-            const int it = b + q * G, bi = q % a.nbuf;
-            const bool is_gu = it < n_gu;
-            int u, p, ks = 0, kd = 0;
-            if (is_gu) {
-                u = it / (P1 * KS);
-                const int r = it % (P1 * KS);
-                p = r / KS;
-                ks = r % KS;
-            } else {
-                const int i2 = it - n_gu;
-                u = i2 / (P2 * 2);
-                const int r = i2 % (P2 * 2);
-                p = r / 2;
-                kd = r % 2;
-            }
-            const int e = act[u], ecnt = cnt[e], eoff = off[e];
-            if (!is_gu) {
-                // every gate/up item of this expert has landed its partial sums
-                bool bad = false;
-                if (tid == 0) bad = !wait_counter(&sync[2 + u], (uint32_t)(P1 * KS), status, &s_abort);
-                if (compute_sync_any(bad || s_abort)) break;
-                const int NS = NT * 8;
-                for (int i = tid; i < NS * FH; i += 512) {  // h = silu(g) * u on this K half, fp16
-                    const int ti = i / FH, c = i % FH;
-                    float h = 0.f;
-                    if (ti < ecnt) {
-                        const int col = kd * FH + c;
-                        float gs = 0.f, us = 0.f;
-                        for (int s2 = 0; s2 < KS; ++s2) {
-                            const size_t base = ((size_t)(s2 * NPD + eoff + ti) * 2) * f + col;
-                            gs += __ldcg(a.ws.gu_part + base);
-                            us += __ldcg(a.ws.gu_part + base + f);
-                        }
-                        h = silu_f(gs) * us;
-                    }
-                    hh[(size_t)ti * dph + c] = __float2half_rn(h);
-                }
-                compute_sync();
-                for (int i = tid; i < NS * (FH / 32); i += 512)
-                    hz[i] = block_constant(hh + (size_t)(i / (FH / 32)) * dph, i % (FH / 32));
-                compute_sync();
-            }
-            const bool landed = mbar_wait(&full[bi], (uint32_t)((q / a.nbuf) & 1), status, &s_abort);
-            if (compute_sync_any(!landed || s_abort)) break;
-            const uint8_t *buf = bufs + (size_t)bi * a.buf_bytes;
-            const int nta = (ecnt + 7) / 8 < NT ? (ecnt + 7) / 8 : NT;
-            const int gr = 16 * rg + g;  // this lane's rows gr and gr + 8 of the panel
-            float out[NT][4];
+            const int u = b + q * G;
+            const int e = act[u / FP];
+            const int ecnt = cnt[e], eoff = off[e];
+            const int nta = min((ecnt + 7) / 8, NT);
+            // ---- gate / up over all of K
+            {
+                float out[RGM][NT][4];
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
+                for (int r = 0; r < RGM; ++r)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) out[n][i] = 0.f;
-            if (is_gu) {
-                const int m = warp >> 3;  // 0 gate, 1 up
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) out[r][n][i] = 0.f;
                 const __half *xb[NT];
                 const float *z0[NT], *z1[NT];
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     const int sb = 8 * n + g, sa = 8 * n + 2 * t4;
-                    const int tb = sb < ecnt ? ptok[eoff + sb] : T;  // T: the zero row
-                    const int ta = sa < ecnt ? ptok[eoff + sa] : T, tc = sa + 1 < ecnt ? ptok[eoff + sa + 1] : T;
-                    xb[n] = xh + (size_t)tb * dpx;
-                    z0[n] = xz + (size_t)ta * (d / 32);
-                    z1[n] = xz + (size_t)tc * (d / 32);
+                    xb[n] = xh + (size_t)(sb < ecnt ? ptok[eoff + sb] : T) * dpx + 2 * t4;  // T: the zero row
+                    z0[n] = xz + (size_t)(sa < ecnt ? ptok[eoff + sa] : T) * (d / 32);
+                    z1[n] = xz + (size_t)(sa + 1 < ecnt ? ptok[eoff + sa + 1] : T) * (d / 32);
                 }
-                for (int sl = 0; sl < SL; ++sl) {
-                    const int col0 = (ks * SL + sl) * 64;
-                    const uint8_t *tile = buf + (size_t)sl * 5120 + m * 2560;
-                    const uint32_t wg = *reinterpret_cast<const uint32_t *>(tile + 16 * gr + 4 * t4);
-                    const uint32_t wg8 = *reinterpret_cast<const uint32_t *>(tile + 16 * (gr + 8) + 4 * t4);
-                    const uint32_t sg = *reinterpret_cast<const uint32_t *>(tile + 2048 + 4 * gr);
-                    const uint32_t sg8 = *reinterpret_cast<const uint32_t *>(tile + 2048 + 4 * (gr + 8));
-                    const __half *xc[NT];
-                    const float *zc0[NT], *zc1[NT];
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        xc[n] = xb[n] + col0;
-                        zc0[n] = z0[n] + col0 / 32;
-                        zc1[n] = z1[n] + col0 / 32;
+                for (int i = 0; i < nG; ++i, ++c) {
+                    const int bi = c % a.nbuf;
+                    if (!bad) bad = !mbar_wait(&full[bi], (uint32_t)((c / a.nbuf) & 1), status, &s_abort);
+                    if (!bad) {
+                        const uint8_t *buf = bufs + (size_t)bi * kChunkBytes;
+                        const int s0 = i * kGuSlicesPerChunk, ns = min(kGuSlicesPerChunk, SLK - s0);
+                        for (int sl = kq; sl < ns; sl += KSPLIT) {
+                            const uint8_t *tiles = buf + (size_t)sl * 2 * kTileBytes;
+                            const int col0 = (s0 + sl) * 64;
+                            if (NT == 1 || nta == 1)
+                                gu_slice<1, NT, RGM, ODD>(tiles, xb, z0, z1, col0, rgm0, g, out);
+                            else
+                                gu_slice<NT, NT, RGM, ODD>(tiles, xb, z0, z1, col0, rgm0, g, out);
+                        }
                     }
-                    tile_mma<NT>(wg, wg8, sg, sg8, xc, zc0, zc1, nta, out);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[bi]);
                 }
+                if (compute_sync_any(bad || s_abort)) {  // every compute warp takes the same branch
+                    stop = true;
+                    break;
+                }
+                // partial sums of this K group: red[kq][matrix][row][slot], slots < TT
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const int sa = 8 * n + 2 * t4;
-                    const size_t col = (size_t)m * f + p * 128 + gr;
-                    if (sa < ecnt) {
-                        float *dst = a.ws.gu_part + ((size_t)(ks * NPD + eoff + sa) * 2) * f + col;
-                        dst[0] = out[n][0];
-                        dst[8] = out[n][2];
-                    }
-                    if (sa + 1 < ecnt) {
-                        float *dst = a.ws.gu_part + ((size_t)(ks * NPD + eoff + sa + 1) * 2) * f + col;
-                        dst[0] = out[n][1];
-                        dst[8] = out[n][3];
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[bi]);  // buffer consumed by this warp
-                compute_sync();
-                if (tid == 0) {  // release the partial sums of this item
-                    __threadfence();
-                    atomicAdd(&sync[2 + u], 1u);
-                }
-            } else {
-                const int half = warp >> 3;  // half of the item's K slices
-                const __half *xb[NT];
-                const float *z0[NT], *z1[NT];
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    xb[n] = hh + (size_t)(8 * n + g) * dph;
-                    z0[n] = hz + (size_t)(8 * n + 2 * t4) * (FH / 32);
-                    z1[n] = hz + (size_t)(8 * n + 2 * t4 + 1) * (FH / 32);
-                }
-                const int s_lo = half * ((SLD + 1) / 2), s_hi = min(SLD, s_lo + (SLD + 1) / 2);
-                for (int sl = s_lo; sl < s_hi; ++sl) {
-                    const uint8_t *tile = buf + (size_t)sl * 2560;
-                    const uint32_t wg = *reinterpret_cast<const uint32_t *>(tile + 16 * gr + 4 * t4);
-                    const uint32_t wg8 = *reinterpret_cast<const uint32_t *>(tile + 16 * (gr + 8) + 4 * t4);
-                    const uint32_t sg = *reinterpret_cast<const uint32_t *>(tile + 2048 + 4 * gr);
-                    const uint32_t sg8 = *reinterpret_cast<const uint32_t *>(tile + 2048 + 4 * (gr + 8));
-                    const __half *xc[NT];
-                    const float *zc0[NT], *zc1[NT];
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        xc[n] = xb[n] + sl * 64;
-                        zc0[n] = z0[n] + sl * 2;
-                        zc1[n] = z1[n] + sl * 2;
-                    }
-                    tile_mma<NT>(wg, wg8, sg, sg8, xc, zc0, zc1, nta, out);
-                }
-                if (s_lo < s_hi) {
+                for (int r = 0; r < RGM; ++r) {
+                    const int rgm = rgm0 + r, m = rgm >> 2, gr = 16 * (rgm & 3) + g;
+                    float *rd = red + (size_t)((kq * 2 + m) * 64) * TT;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         const int sa = 8 * n + 2 * t4;
-                        const int row = p * 128 + gr;
-                        if (sa < ecnt) {
-                            float *yr = a.y + (size_t)ptok[eoff + sa] * d + row;
-                            atomicAdd(yr, pw[eoff + sa] * out[n][0]);
-                            atomicAdd(yr + 8, pw[eoff + sa] * out[n][2]);
+                        if (sa < TT) {
+                            rd[gr * TT + sa] = out[r][n][0];
+                            rd[(gr + 8) * TT + sa] = out[r][n][2];
                         }
-                        if (sa + 1 < ecnt) {
-                            float *yr = a.y + (size_t)ptok[eoff + sa + 1] * d + row;
-                            atomicAdd(yr, pw[eoff + sa + 1] * out[n][1]);
-                            atomicAdd(yr + 8, pw[eoff + sa + 1] * out[n][3]);
+                        if (sa + 1 < TT) {
+                            rd[gr * TT + sa + 1] = out[r][n][1];
+                            rd[(gr + 8) * TT + sa + 1] = out[r][n][3];
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[bi]);
             }
+            compute_sync();
+            // ---- h = silu(g) * u for the slice's 64 rows (fp16) and its block constants
+            for (int i = tid; i < NS * 64; i += 512) {
+                const int slot = i / 64, row = i % 64;
+                float h = 0.f;
+                if (slot < ecnt) {
+                    float gs = 0.f, us = 0.f;
+#pragma unroll
+                    for (int kg = 0; kg < KSPLIT; ++kg) {
+                        gs += red[((kg * 2 + 0) * 64 + row) * TT + slot];
+                        us += red[((kg * 2 + 1) * 64 + row) * TT + slot];
+                    }
+                    h = silu_f(gs) * us;
+                }
+                hh[slot * kHStride + row] = __float2half_rn(h);
+            }
+            compute_sync();
+            if (warp < NS) row_block_constants(hh + warp * kHStride, 64, hz + warp * 2);
+            compute_sync();
+            // ---- down: y[token] += w * W_down[:, slice] h
+            {
+                uint32_t bf[NT][4][2];
+                float zf[NT][2][2];
+                int tokA[NT], tokB[NT];
+                float wA[NT], wB[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const __half *hr = hh + (8 * n + g) * kHStride + 2 * t4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        bf[n][j][0] = *reinterpret_cast<const uint32_t *>(hr + 16 * j);
+                        bf[n][j][1] = *reinterpret_cast<const uint32_t *>(hr + 16 * j + 8);
+                    }
+                    const int sa = 8 * n + 2 * t4;
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        zf[n][blk][0] = hz[sa * 2 + blk];
+                        zf[n][blk][1] = hz[(sa + 1) * 2 + blk];
+                    }
+                    tokA[n] = sa < ecnt ? ptok[eoff + sa] : -1;
+                    tokB[n] = sa + 1 < ecnt ? ptok[eoff + sa + 1] : -1;
+                    wA[n] = sa < ecnt ? pw[eoff + sa] : 0.f;
+                    wB[n] = sa + 1 < ecnt ? pw[eoff + sa + 1] : 0.f;
+                }
+                for (int i = 0; i < nD; ++i, ++c) {
+                    const int bi = c % a.nbuf;
+                    if (!bad) bad = !mbar_wait(&full[bi], (uint32_t)((c / a.nbuf) & 1), status, &s_abort);
+                    if (!bad) {
+                        const uint8_t *buf = bufs + (size_t)bi * kChunkBytes;
+                        const int p0 = i * kDownPanelsPerChunk, np = min(kDownPanelsPerChunk, SLK - p0);
+                        for (int rgi = warp; rgi < np * 4; rgi += kFusedComputeWarps) {
+                            const int pan = rgi >> 2, r16 = 16 * (rgi & 3) + g;
+                            const TileRows w = load_rows(buf + (size_t)pan * kTileBytes, r16);
+                            float o[NT][4];
+#pragma unroll
+                            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                                for (int z = 0; z < 4; ++z) o[n][z] = 0.f;
+                            if (NT == 1 || nta == 1)
+                                down_rows<1, NT, ODD>(w, bf, zf, o);
+                            else
+                                down_rows<NT, NT, ODD>(w, bf, zf, o);
+                            const int row = (p0 + pan) * 64 + r16;
+#pragma unroll
+                            for (int n = 0; n < NT; ++n) {
+                                if (tokA[n] >= 0) {
+                                    float *yr = a.y + (size_t)tokA[n] * d + row;
+                                    atomicAdd(yr, wA[n] * o[n][0]);
+                                    atomicAdd(yr + 8, wA[n] * o[n][2]);
+                                }
+                                if (tokB[n] >= 0) {
+                                    float *yr = a.y + (size_t)tokB[n] * d + row;
+                                    atomicAdd(yr, wB[n] * o[n][1]);
+                                    atomicAdd(yr + 8, wB[n] * o[n][3]);
+                                }
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[bi]);
+                }
+            }
+            // a failed copy wait in the down chunks reaches the other warps
+            // at the next unit's first barrier, or at the one below
         }
+        // Either every compute warp left the loop through the barrier above
+        // (stop), or none did and all of them meet here once.
+        if (!stop) compute_sync_any(bad);
     }
     // the last CTA out clears the counters for the next launch
     __syncthreads();
@@ -755,7 +887,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         const uint32_t prev = atomicAdd(&sync[1], 1u);
         if (prev == (uint32_t)G - 1) {
             sync[0] = 0;
-            for (int i = 0, n = s_abort ? E : n_act; i < n; ++i) sync[2 + i] = 0;
             __threadfence();
             sync[1] = 0;
         }
@@ -764,40 +895,74 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
 
 // ---------------------------------------------------------------- host side
 struct FusedConfig {
-    int KS, nbuf;
-    uint32_t buf_bytes;
+    int nbuf;
     size_t smem;
 };
+
+// Measured on B200: when a block's shared memory forces the largest
+// shared-memory carveout (L1 left with about 28 KB), the MMA loops run about
+// 40% slower than with 150 KB of shared memory. The ring is therefore sized
+// to stay under kFusedSmemSoftCap when that still leaves kFusedMinRing
+// chunks, and only otherwise grows to the device limit.
+constexpr long long kFusedSmemSoftCap = 150 * 1024;
+constexpr int kFusedMinRing = 4;
 
 static FusedConfig fused_config(const Shape &s, int T, int max_smem) {
     FusedConfig c;
     const int TT = T <= 1 ? 1 : T <= 4 ? 4 : 16;
-    c.KS = 4;
-    while (c.KS > 1 && (s.d / 64) % c.KS) c.KS /= 2;
-    const uint32_t gu = (uint32_t)((s.d / 64) / c.KS) * 5120u;
-    const uint32_t dn = (uint32_t)((s.f / 2) / 64) * 2560u;
-    c.buf_bytes = (gu > dn ? gu : dn);
-    c.buf_bytes = (c.buf_bytes + 127) & ~127u;
-    const FusedSmem base = fused_plan(T, TT, s.d, s.f, s.E, s.k, 0, c.buf_bytes);
-    const long long room = (long long)max_smem - 2048 - (long long)base.total;
-    c.nbuf = room > 0 ? (int)(room / c.buf_bytes) : 0;
-    if (c.nbuf > kFusedMaxBuf) c.nbuf = kFusedMaxBuf;
-    c.smem = fused_plan(T, TT, s.d, s.f, s.E, s.k, c.nbuf, c.buf_bytes).total;
+    const FusedSmem base = fused_plan(T, TT, s.d, s.E, s.k, 0);
+    auto ring = [&](long long limit) {
+        const long long room = limit - 2048 - (long long)base.total;
+        const int n = room > 0 ? (int)(room / kChunkBytes) : 0;
+        return n > kFusedMaxBuf ? kFusedMaxBuf : n;
+    };
+    c.nbuf = ring(kFusedSmemSoftCap < max_smem ? kFusedSmemSoftCap : max_smem);
+    if (c.nbuf < kFusedMinRing) c.nbuf = ring(max_smem);
+    c.smem = fused_plan(T, TT, s.d, s.E, s.k, c.nbuf).total;
     return c;
 }
 
-bool decode_fused_supported(const Shape &s, int T, int max_smem) {
-    // one candidate scan per lane holds at most 1024 experts per warp; two
-    // experts per compute thread in the count scans
-    if (T < 1 || T > kDecMaxT || (s.f / 2) % 64 || s.E > 1024) return false;
+bool decode_fused_supported(const Shape &s, int T, int max_smem, int num_sms) {
+    // one warp per token in the routing, 16 logits per lane read 4 at a
+    // time; at most kRouterRowsMax router rows per CTA; 64-column tiles on
+    // both sides of every matrix
+    if (T < 1 || T > kDecMaxT || s.E > 512 || s.E % 4 || s.d % 64 || s.f % 64) return false;
+    if (num_sms < 1 || (s.E + num_sms - 1) / num_sms > kRouterRowsMax) return false;
     return fused_config(s, T, max_smem).nbuf >= 2;
 }
 
-cudaError_t init_fused_attributes(int max_smem) {
-    cudaError_t e = set_max_dynamic_smem(k_decode_fused<1>, max_smem);
-    if (e == cudaSuccess) e = set_max_dynamic_smem(k_decode_fused<4>, max_smem);
-    if (e == cudaSuccess) e = set_max_dynamic_smem(k_decode_fused<16>, max_smem);
+// The kernels' shared-memory limit is raised only as far as the launches
+// need: a larger limit makes the driver pick a larger shared-memory carveout
+// (less L1), which slows the MMA loops (see kFusedSmemSoftCap). Kept per
+// device and instantiation; raised at layer creation, before any capture.
+static std::mutex g_limit_mutex;
+static int g_limit[64][3];
+
+static cudaError_t ensure_limit(int slot, int need) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_limit_mutex);
+    if (g_limit[dev][slot] >= need) return cudaSuccess;
+    if (slot == 0) e = cudaFuncSetAttribute(k_decode_fused<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+    if (slot == 1) e = cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+    if (slot == 2) e = cudaFuncSetAttribute(k_decode_fused<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+    if (e == cudaSuccess) g_limit[dev][slot] = need;
     return e;
+}
+
+static int slot_of(int T) { return T <= 1 ? 0 : T <= 4 ? 1 : 2; }
+
+cudaError_t init_fused_attributes(const Shape &s, int max_tokens, int max_smem, int num_sms) {
+    static const int tts[3] = {1, 4, 16};
+    for (int i = 0; i < 3; ++i) {
+        const int T = tts[i] < max_tokens ? tts[i] : max_tokens;
+        if (slot_of(T) != i || !decode_fused_supported(s, T, max_smem, num_sms)) continue;
+        const cudaError_t e = ensure_limit(i, (int)fused_config(s, T, max_smem).smem);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float *W, const float *bias,
@@ -820,9 +985,8 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
     a.eps = eps;
     a.ebytes = expert_bytes(s);
     a.down_off = down_section_offset(s);
-    a.KS = c.KS;
+    a.xs = expert_strides(s);
     a.nbuf = c.nbuf;
-    a.buf_bytes = c.buf_bytes;
     a.ws = ws;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms);
@@ -834,8 +998,9 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cudaError_t e = ensure_limit(slot_of(T), (int)c.smem);  // a no-op after layer creation
+    if (e != cudaSuccess) return e;
     if (ev) cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal);
-    cudaError_t e;
     if (T <= 1)
         e = cudaLaunchKernelEx(&cfg, k_decode_fused<1>, a);
     else if (T <= 4)

@@ -24,14 +24,13 @@ struct Workspace {
     int32_t *pair_of;     // [T * k]   (t, j) -> index in the sorted pair list
     int32_t *blk_counts;  // [nblk * E] per 256-token block (prefill lists)
     int32_t *act;         // [E] active experts (decode path)
-    float *gu_part;       // [KS * Pd * 2 * f]   fused decode: gate/up partial sums
-    float *lpart;         // [16 * E * 4]        fused decode: router partial sums
+    float *lpart;         // [16 * E * 4]        fused decode: router logits [T][E]
     void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill)
     void *hbuf;           // fp16 [T*k * f]       SwiGLU outputs (prefill)
     int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
     int4 *tiles2;         // down GEMM tiles
     void *xn;             // bf16 [T * d]         stack: normalised input
-    uint32_t *sync;       // [2 + E] fused decode: grid barrier, exit count, per-expert gate/up counters
+    uint32_t *sync;       // [2]     fused decode: grid barrier, exit count
 };
 
 // meta[] slots
@@ -39,7 +38,6 @@ enum { META_N_ACTIVE = 0, META_N_TILES1 = 1, META_N_TILES2 = 2, META_N_TOKENS = 
 
 constexpr int kRouteBlock = 256;      // tokens per block of the prefill lists
 constexpr int kDecMaxT = 16;          // largest token count of the streaming path
-constexpr int kDecKS = 4;             // fused decode gate/up K splits (max)
 constexpr int kGemm1N = 128;          // gate/up GEMM: max tokens per tile
 constexpr int kGemm2N = 256;          // down GEMM: max tokens per tile
 
@@ -61,8 +59,9 @@ void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tile
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st);
 
 // --- fused decode layer (T <= 16, one cooperative launch)
-bool decode_fused_supported(const Shape &s, int T, int max_smem);
-cudaError_t init_fused_attributes(int max_smem);
+bool decode_fused_supported(const Shape &s, int T, int max_smem, int num_sms);
+// raise the kernels' shared-memory limits to what this shape needs (layer creation)
+cudaError_t init_fused_attributes(const Shape &s, int max_tokens, int max_smem, int num_sms);
 cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float *W, const float *bias,
                                 const uint8_t *blob, float *y, bool accumulate, bool rms, float eps, int T,
                                 const Shape &s, int num_sms, int max_smem, cudaStream_t st, cudaEvent_t *ev);
@@ -76,10 +75,26 @@ void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, con
 // --- misc
 void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cudaStream_t st);
 void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
-                               size_t tile_stride, cudaStream_t st);
+                               size_t panel_stride, size_t slice_stride, cudaStream_t st);
 void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st);
 
 size_t expert_bytes(const Shape &s);
+
+// Q2 tiles: 64 rows x 64 columns, codes then scales.
+constexpr int kTileRows = 64;
+constexpr int kTileBytes = 1280;
+constexpr int kTileScaleOffset = 1024;
+
+// Byte strides between the tiles of an expert's matrices: gate/up tiles
+// (f-panel p, d-slice s) at p * gu_panel + s * gu_slice (gate, then up at
+// +1280); down tiles (d-panel p, f-slice s) at p * dn_panel + s * dn_slice.
+struct ExpertStrides {
+    size_t gu_panel, gu_slice, dn_panel, dn_slice;
+};
+inline ExpertStrides expert_strides(const Shape &s) {
+    return ExpertStrides{(size_t)(s.d / 64) * 2 * kTileBytes, (size_t)2 * kTileBytes, (size_t)kTileBytes,
+                         (size_t)(s.d / 64) * kTileBytes};
+}
 
 // Allow `kernel` the largest dynamic shared memory the device grants a block
 // (max_total, the opt-in limit) minus its static shared memory.

@@ -36,17 +36,17 @@ void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cud
 // ------------------------------------------------------------ packer
 // One thread per (tile, row): 64 codes -> four words (column
 // c = 16j + 8s + 2t + h in word t at bit 16h + 8s + 6 - 2j), then the row's
-// two block scales.
+// two block scales. Tile (p, s) goes to dst + p * panel_stride + s * slice_stride.
 __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales, int rows, int K,
-                              uint8_t *__restrict__ dst, size_t tile_stride) {
+                              uint8_t *__restrict__ dst, size_t panel_stride, size_t slice_stride) {
     const int slices = K / 64;
-    const long long n = (long long)(rows / 128) * slices * 128;
+    const long long n = (long long)(rows / kTileRows) * slices * kTileRows;
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= n) return;
-    const int i = (int)(g & 127);
-    const long long tile = g >> 7;
+    const int i = (int)(g % kTileRows);
+    const long long tile = g / kTileRows;
     const int p = (int)(tile / slices), s = (int)(tile % slices);
-    const int r = p * 128 + i;
+    const int r = p * kTileRows + i;
     const uint8_t *cr = codes + (size_t)r * K + (size_t)s * 64;
     uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll 4
@@ -54,17 +54,18 @@ __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t 
         const uint32_t v = cr[c] & 3u;
         w[(c & 7) >> 1] |= v << (16 * (c & 1) + 8 * ((c >> 3) & 1) + 6 - 2 * (c >> 4));
     }
-    uint8_t *t = dst + (size_t)tile * tile_stride;
+    uint8_t *t = dst + (size_t)p * panel_stride + (size_t)s * slice_stride;
     *reinterpret_cast<uint4 *>(t + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
     const uint16_t *sr = scales + (size_t)r * (K / 32) + 2 * s;
-    *reinterpret_cast<uint32_t *>(t + 2048 + 4 * i) = (uint32_t)sr[0] | ((uint32_t)sr[1] << 16);
+    *reinterpret_cast<uint32_t *>(t + kTileScaleOffset + 4 * i) = (uint32_t)sr[0] | ((uint32_t)sr[1] << 16);
 }
 
 void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
-                               size_t tile_stride, cudaStream_t st) {
-    const long long n = (long long)(rows / 128) * (K / 64) * 128;
+                               size_t panel_stride, size_t slice_stride, cudaStream_t st) {
+    const long long n = (long long)(rows / kTileRows) * (K / 64) * kTileRows;
     if (n <= 0) return;
-    k_pack_matrix<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(codes, scales, rows, K, dst, tile_stride);
+    k_pack_matrix<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(codes, scales, rows, K, dst, panel_stride,
+                                                                slice_stride);
 }
 
 // ------------------------------------------------------------ self test

@@ -4,8 +4,8 @@
 // Prompts are read in chunks of up to 8,192 tokens and the expert products
 // run on the quantised weights instead of first expanding them to FP16 in
 // memory ("Strata：把 125B 大模型塞进 12GB 显卡…", 工程细节). Here every
-// 128-row x 64-column tile of 2-bit weights is copied once per token tile
-// into shared memory (1-D bulk copy), dequantised there to fp16, and fed to
+// 128-row x 64-column block of 2-bit weights (two 64-row tiles) is copied once
+// per token tile into shared memory (1-D bulk copies), dequantised there to fp16, and fed to
 // tcgen05.mma; the tokens of one expert (a contiguous run of the gathered,
 // expert-sorted rows) come in by 2-D tensor copies with 128-byte swizzle.
 //
@@ -45,7 +45,7 @@ struct GLayout {
     static constexpr int NMAT = GCfg<MODE>::NMAT, NMAX = GCfg<MODE>::NMAX, STAGES = GCfg<MODE>::STAGES;
     static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // one fp16 matrix tile
     static constexpr uint32_t B_BYTES = NMAX * 128;    // NMAX rows of 64 fp16
-    static constexpr uint32_t W_BYTES = NMAT * 2560;   // packed 2-bit tile(s)
+    static constexpr uint32_t W_BYTES = NMAT * 2 * kTileBytes;  // packed 2-bit tiles: 128 rows per matrix
     static constexpr uint32_t STAGE = ((NMAT * A_BYTES + B_BYTES + W_BYTES) + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM = STAGES * STAGE + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -56,6 +56,8 @@ struct GemmArgs {
     const uint8_t *blob;
     size_t ebytes;     // bytes per expert
     size_t sec_off;    // byte offset of this GEMM's section inside an expert
+    size_t tile_panel; // byte stride between 64-row tile panels of the section
+    size_t tile_slice; // byte stride between 64-column K slices of the section
     int K;             // reduction length (d for MODE 0, f for MODE 1)
     int panels;        // 128-row panels of the output (f/128 or d/128)
     int ldo;           // MODE 0: f (row length of H); MODE 1: d (row length of y)
@@ -121,8 +123,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                 const int npad = (tl.z + 15) & ~15;
                 const int bsel = npad <= 16 ? 0 : npad <= 32 ? 1 : npad <= 64 ? 2 : npad <= 128 ? 3 : 4;
                 const uint32_t brows = 16u << bsel;
-                const uint8_t *wsrc = a.blob + (size_t)tl.x * a.ebytes + a.sec_off +
-                                      (size_t)panel * KSTEPS * L::W_BYTES;
+                const uint8_t *wsrc = a.blob + (size_t)tl.x * a.ebytes + a.sec_off + (size_t)(2 * panel) * a.tile_panel;
                 bool ok = true;
                 for (int ks = 0; ks < KSTEPS; ++ks, ++it) {
                     const int st = it % S;
@@ -132,7 +133,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                         break;
                     }
                     mbar_arrive_expect_tx(&full[st], L::W_BYTES + brows * 128);
-                    bulk_g2s(W_at(st), wsrc + (size_t)ks * L::W_BYTES, L::W_BYTES, &full[st]);
+                    if (MODE == 0) {  // (gate, up) pairs of the panel's two 64-row halves
+                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * kTileBytes, &full[st]);
+                        bulk_g2s(W_at(st) + 2 * kTileBytes, wsrc + a.tile_panel + (size_t)ks * a.tile_slice,
+                                 2 * kTileBytes, &full[st]);
+                    } else {  // the two 64-row tiles of a down panel are adjacent
+                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * kTileBytes, &full[st]);
+                    }
                     tma_load_2d(B_at(st), &maps.m[bsel], ks * 64, tl.y, &full[st]);
                 }
                 if (!ok) break;
@@ -235,9 +242,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     ok = false;
                     break;
                 }
-                const uint8_t *wt = W_at(st) + mat * 2560;
-                const uint4 cw = *reinterpret_cast<const uint4 *>(wt + 16 * row);
-                uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + 2048 + 4 * row);
+                // row r of the 128-row block: tile half r / 64, row r % 64 of that tile
+                const uint8_t *wt = W_at(st) + (row >> 6) * (NMAT * kTileBytes) + mat * kTileBytes;
+                const int ri = row & 63;
+                const uint4 cw = *reinterpret_cast<const uint4 *>(wt + 16 * ri);
+                uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + kTileScaleOffset + 4 * ri);
                 const __half2 s01 = __hmul2(*reinterpret_cast<__half2 *>(&scb), khalf);  // (s0/2, s1/2)
                 const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -295,6 +304,8 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
     a.blob = blob;
     a.ebytes = expert_bytes(s);
     a.sec_off = 0;
+    a.tile_panel = expert_strides(s).gu_panel;
+    a.tile_slice = expert_strides(s).gu_slice;
     a.K = s.d;
     a.panels = s.f / 128;
     a.ldo = s.f;
@@ -312,6 +323,8 @@ void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, con
     a.blob = blob;
     a.ebytes = expert_bytes(s);
     a.sec_off = down_section_offset(s);
+    a.tile_panel = expert_strides(s).dn_panel;
+    a.tile_slice = expert_strides(s).dn_slice;
     a.K = s.f;
     a.panels = s.d / 128;
     a.ldo = s.d;

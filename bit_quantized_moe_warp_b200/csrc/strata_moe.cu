@@ -102,7 +102,7 @@ static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
-    size_t off[21];
+    size_t off[20];
     size_t total;
     int max_tiles1, max_tiles2;
 };
@@ -111,12 +111,11 @@ static Plan plan_workspace(const strata_moe_desc *d) {
     const Shape s = shape_of(d);
     const size_t T = (size_t)d->max_tokens, k = s.k, E = s.E;
     const size_t P = T * k;
-    const size_t Pd = (size_t)kDecMaxT * k;
     const size_t nblk = (T + kRouteBlock - 1) / kRouteBlock;
     Plan p{};
     p.max_tiles1 = (int)((P + kGemm1N - 1) / kGemm1N + E);
     p.max_tiles2 = (int)((P + kGemm2N - 1) / kGemm2N + E);
-    const size_t sz[21] = {
+    const size_t sz[20] = {
         256,                                      // 0 status
         64 * 4,                                   // 1 meta
         T * E * 4,                                // 2 logits
@@ -130,17 +129,16 @@ static Plan plan_workspace(const strata_moe_desc *d) {
         P * 4,                                    // 10 pair_of
         nblk * E * 4,                             // 11 blk_counts
         E * 4,                                    // 12 act
-        (size_t)kDecKS * Pd * 2 * s.f * 4,        // 13 gu_part
-        (size_t)kDecMaxT * E * 4 * 4,             // 14 lpart
-        P * (size_t)s.d * 2,                      // 15 xp
-        P * (size_t)s.f * 2,                      // 16 hbuf
-        (size_t)p.max_tiles1 * 16,                // 17 tiles1
-        (size_t)p.max_tiles2 * 16,                // 18 tiles2
-        T * (size_t)s.d * 2,                      // 19 xn
-        (2 + E) * 4,                              // 20 sync
+        (size_t)kDecMaxT * E * 4 * 4,             // 13 lpart
+        P * (size_t)s.d * 2,                      // 14 xp
+        P * (size_t)s.f * 2,                      // 15 hbuf
+        (size_t)p.max_tiles1 * 16,                // 16 tiles1
+        (size_t)p.max_tiles2 * 16,                // 17 tiles2
+        T * (size_t)s.d * 2,                      // 18 xn
+        (2 + E) * 4,                              // 19 sync
     };
     size_t o = 0;
-    for (int i = 0; i < 21; ++i) {
+    for (int i = 0; i < 20; ++i) {
         p.off[i] = o;
         o += (sz[i] + 255) & ~(size_t)255;
     }
@@ -163,14 +161,13 @@ static Workspace carve(uint8_t *base, const Plan &p) {
     w.pair_of = reinterpret_cast<int32_t *>(base + p.off[10]);
     w.blk_counts = reinterpret_cast<int32_t *>(base + p.off[11]);
     w.act = reinterpret_cast<int32_t *>(base + p.off[12]);
-    w.gu_part = reinterpret_cast<float *>(base + p.off[13]);
-    w.lpart = reinterpret_cast<float *>(base + p.off[14]);
-    w.xp = base + p.off[15];
-    w.hbuf = base + p.off[16];
-    w.tiles1 = reinterpret_cast<int4 *>(base + p.off[17]);
-    w.tiles2 = reinterpret_cast<int4 *>(base + p.off[18]);
-    w.xn = base + p.off[19];
-    w.sync = reinterpret_cast<uint32_t *>(base + p.off[20]);
+    w.lpart = reinterpret_cast<float *>(base + p.off[13]);
+    w.xp = base + p.off[14];
+    w.hbuf = base + p.off[15];
+    w.tiles1 = reinterpret_cast<int4 *>(base + p.off[16]);
+    w.tiles2 = reinterpret_cast<int4 *>(base + p.off[17]);
+    w.xn = base + p.off[18];
+    w.sync = reinterpret_cast<uint32_t *>(base + p.off[19]);
     return w;
 }
 
@@ -212,11 +209,11 @@ static strata_status make_maps(TmaMaps &m, void *base, size_t rows, int K) {
 
 namespace strata {
 cudaError_t init_gemm_attributes(int max_smem);
-static cudaError_t init_kernel_attributes(int device) {
+static cudaError_t init_kernel_attributes(int device, const Shape &s, int max_tokens, int num_sms) {
     int max_smem = 0;
     cudaError_t e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     if (e == cudaSuccess) e = init_gemm_attributes(max_smem);
-    if (e == cudaSuccess) e = init_fused_attributes(max_smem);
+    if (e == cudaSuccess) e = init_fused_attributes(s, max_tokens, max_smem, num_sms);
     return e;
 }
 }  // namespace strata
@@ -265,7 +262,7 @@ extern "C" strata_status strata_moe_set_stage_events(strata_moe_layer L, void *c
 }
 
 extern "C" size_t strata_q2_matrix_bytes(int32_t rows, int32_t K) {
-    if (rows <= 0 || K <= 0 || rows % 128 || K % 64) return 0;
+    if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS) return 0;
     return (size_t)rows * K / 64 * 20;
 }
 
@@ -343,7 +340,7 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
         int max_smem = 0;
         cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, L->device);
         const int Tw = desc->max_tokens < kDecMaxT ? desc->max_tokens : kDecMaxT;
-        L->fused_ok = decode_fused_supported(L->shape, Tw, max_smem);
+        L->fused_ok = decode_fused_supported(L->shape, Tw, max_smem, L->num_sms);
         L->max_smem = max_smem;
     }
     if (cudaMemset(L->ws.sync, 0, (size_t)(2 + L->shape.E) * 4) != cudaSuccess) {
@@ -351,7 +348,7 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
         delete L;
         return fail(STRATA_ERR_CUDA, "workspace clear failed");
     }
-    if (cudaError_t e = init_kernel_attributes(L->device)) {
+    if (cudaError_t e = init_kernel_attributes(L->device, L->shape, desc->max_tokens, L->num_sms)) {
         cudaGetLastError();
         if (L->owns_ws) cudaFree(L->ws_mem);
         delete L;
@@ -635,14 +632,15 @@ extern "C" strata_status strata_selftest_wait_timeout(uint64_t timeout_ns, strat
 }
 
 // ------------------------------------------------------------ packers
+// Tile (p, s) of a [rows x K] matrix -- rows 64p.., columns 64s.. -- goes to
+// dst + p * panel_stride + s * slice_stride.
 static void pack_matrix_host(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
-                             size_t tile_stride) {
-    const int slices = K / 64;
-    for (int p = 0; p < rows / 128; ++p)
-        for (int s = 0; s < slices; ++s) {
-            uint8_t *t = dst + ((size_t)p * slices + s) * tile_stride;
-            for (int i = 0; i < 128; ++i) {
-                const int r = p * 128 + i;
+                             size_t panel_stride, size_t slice_stride) {
+    for (int p = 0; p < rows / STRATA_Q2_TILE_ROWS; ++p)
+        for (int s = 0; s < K / STRATA_Q2_TILE_COLS; ++s) {
+            uint8_t *t = dst + (size_t)p * panel_stride + (size_t)s * slice_stride;
+            for (int i = 0; i < STRATA_Q2_TILE_ROWS; ++i) {
+                const int r = p * STRATA_Q2_TILE_ROWS + i;
                 uint32_t w[4] = {0, 0, 0, 0};
                 for (int c = 0; c < 64; ++c)  // c = 16j + 8s + 2t + h -> word t, bit 16h + 8s + 6 - 2j
                     w[(c % 8) / 2] |= (uint32_t)(codes[(size_t)r * K + 64 * s + c] & 3u)
@@ -651,8 +649,8 @@ static void pack_matrix_host(const uint8_t *codes, const uint16_t *scales, int r
                     for (int b = 0; b < 4; ++b) t[16 * i + 4 * q + b] = (uint8_t)(w[q] >> (8 * b));
                 for (int b = 0; b < 2; ++b) {
                     const uint16_t sv = scales[(size_t)r * (K / 32) + 2 * s + b];
-                    t[2048 + 4 * i + 2 * b] = (uint8_t)(sv & 0xff);
-                    t[2048 + 4 * i + 2 * b + 1] = (uint8_t)(sv >> 8);
+                    t[kTileScaleOffset + 4 * i + 2 * b] = (uint8_t)(sv & 0xff);
+                    t[kTileScaleOffset + 4 * i + 2 * b + 1] = (uint8_t)(sv >> 8);
                 }
             }
         }
@@ -667,11 +665,12 @@ static strata_status check_codes(const uint8_t *codes, size_t n) {
 extern "C" strata_status strata_q2_pack(const uint8_t *codes, const uint16_t *scales, int32_t rows, int32_t K,
                                         void *dst) {
     if (!codes || !scales || !dst) return fail(STRATA_ERR_INVALID_ARG, "NULL pointer");
-    if (rows <= 0 || K <= 0 || rows % 128 || K % 64)
-        return fail(STRATA_ERR_INVALID_ARG, "rows must be a multiple of 128 and K of 64 (got %d x %d)", rows, K);
+    if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS)
+        return fail(STRATA_ERR_INVALID_ARG, "rows and K must be multiples of 64 (got %d x %d)", rows, K);
     strata_status s = check_codes(codes, (size_t)rows * K);
     if (s != STRATA_OK) return s;
-    pack_matrix_host(codes, scales, rows, K, static_cast<uint8_t *>(dst), STRATA_Q2_TILE_BYTES);
+    pack_matrix_host(codes, scales, rows, K, static_cast<uint8_t *>(dst),
+                     (size_t)(K / STRATA_Q2_TILE_COLS) * STRATA_Q2_TILE_BYTES, STRATA_Q2_TILE_BYTES);
     return STRATA_OK;
 }
 
@@ -687,9 +686,10 @@ extern "C" strata_status strata_moe_pack_expert(const strata_moe_desc *desc, con
         (s = check_codes(dc, n)) != STRATA_OK)
         return s;
     uint8_t *b = static_cast<uint8_t *>(dst);
-    pack_matrix_host(gc, gs, sh.f, sh.d, b, 2 * STRATA_Q2_TILE_BYTES);
-    pack_matrix_host(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, 2 * STRATA_Q2_TILE_BYTES);
-    pack_matrix_host(dc, ds, sh.d, sh.f, b + down_section_offset(sh), STRATA_Q2_TILE_BYTES);
+    const ExpertStrides x = expert_strides(sh);
+    pack_matrix_host(gc, gs, sh.f, sh.d, b, x.gu_panel, x.gu_slice);
+    pack_matrix_host(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, x.gu_panel, x.gu_slice);
+    pack_matrix_host(dc, ds, sh.d, sh.f, b + down_section_offset(sh), x.dn_panel, x.dn_slice);
     return STRATA_OK;
 }
 
@@ -704,8 +704,9 @@ extern "C" strata_status strata_moe_pack_expert_device(const strata_moe_desc *de
     const Shape sh = shape_of(desc);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *b = static_cast<uint8_t *>(dst);
-    launch_pack_matrix_device(gc, gs, sh.f, sh.d, b, 2 * STRATA_Q2_TILE_BYTES, st);
-    launch_pack_matrix_device(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, 2 * STRATA_Q2_TILE_BYTES, st);
-    launch_pack_matrix_device(dc, ds, sh.d, sh.f, b + down_section_offset(sh), STRATA_Q2_TILE_BYTES, st);
+    const ExpertStrides x = expert_strides(sh);
+    launch_pack_matrix_device(gc, gs, sh.f, sh.d, b, x.gu_panel, x.gu_slice, st);
+    launch_pack_matrix_device(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, x.gu_panel, x.gu_slice, st);
+    launch_pack_matrix_device(dc, ds, sh.d, sh.f, b + down_section_offset(sh), x.dn_panel, x.dn_slice, st);
     return check_launch("pack kernels");
 }

@@ -62,9 +62,9 @@ typedef enum {
  * page, 功能与原则; its bits are this library's).
  *   weight W[r][k] = (c[r][k] - 1.5) * s[r][k/32], c in {0,1,2,3}, s fp16:
  *   32-weight blocks along the reduction dimension K of each output row.
- * A matrix [R x K] (R % 128 == 0, K % 64 == 0) is a sequence of tiles, one
- * per (128-row panel p, 64-column slice s); a tile is 2560 bytes:
- *   bytes [0, 2048):   codes, row i (0..127) at bytes 16i..16i+15, as four
+ * A matrix [R x K] (R % 64 == 0, K % 64 == 0) is stored as tiles, one per
+ * (64-row panel p, 64-column slice s); a tile is 1280 bytes:
+ *   bytes [0, 1024):   codes, row i (0..63) at bytes 16i..16i+15, as four
  *                      little-endian uint32 words W0..W3; column c (0..63)
  *                      of the tile, written c = 16j + 8s + 2t + h (j < 4,
  *                      s < 2, t < 4, h < 2), lives in word Wt at bit
@@ -74,23 +74,28 @@ typedef enum {
  *                      (columns 2t, 2t+1, 2t+8, 2t+9 of each 16-column
  *                      step), and one mask per register extracts the two
  *                      codes of a column pair without a shift;
- *   bytes [2048, 2560): scales, row i at 2048+4i: fp16 (little-endian) of
+ *   bytes [1024, 1280): scales, row i at 1024+4i: fp16 (little-endian) of
  *                      block 2s, then of block 2s+1.
  * Every tile is a multiple of 16 bytes, so tiles serve 128-bit loads and
- * 1-D bulk (TMA) copies alike; a 64-column slice of a 128-row panel, as the
- * tensor-core path consumes it, is one contiguous tile.
+ * 1-D bulk (TMA) copies alike. A lone matrix (strata_q2_pack) keeps its
+ * tiles in (p, s) order: tile (p, s) at byte (p * K/64 + s) * 1280.
  *
  * Expert blob: experts 0..E-1 back to back, strata_moe_expert_bytes() each:
- *   gate/up section: for p in 0..f/128-1, for s in 0..d/64-1:
- *                    [gate tile (p,s)][up tile (p,s)]     (5120 bytes)
- *   down section:    down matrix [d x f] tiles in (p, s) order, p < d/128,
- *                    s < f/64                              (2560 bytes each)
+ *   gate/up section: for p in 0..f/64-1, for s in 0..d/64-1:
+ *                    [gate tile (p,s)][up tile (p,s)]     (2560 bytes)
+ *   down section:    down matrix [d x f], for s in 0..f/64-1 (its K slices),
+ *                    for p in 0..d/64-1: tile (p,s)       (1280 bytes each)
  *   per expert: 3*d*f/32*10 bytes (d=2048, f=768: 1,474,560 bytes).
+ * The order keeps, contiguous in memory, everything one 64-row slice of the
+ * expert's hidden layer needs: its gate and up rows over all of K
+ * ((d/64) * 2560 bytes) and the down columns it feeds ((d/64) * 1280
+ * bytes); the tensor-core path's 128-row panels are two adjacent 64-row
+ * tiles (down) or two 2560-byte pairs (gate/up).
  */
 #define STRATA_FMT_Q2_0_TILED 1
-#define STRATA_Q2_TILE_ROWS 128
+#define STRATA_Q2_TILE_ROWS 64
 #define STRATA_Q2_TILE_COLS 64
-#define STRATA_Q2_TILE_BYTES 2560
+#define STRATA_Q2_TILE_BYTES 1280
 
 /* desc.flags */
 #define STRATA_ACCUMULATE 1u      /* y += MoE(x) instead of y = MoE(x) */
@@ -113,7 +118,7 @@ typedef struct {
 
 typedef struct strata_moe_layer_s *strata_moe_layer;
 
-/* Bytes of one packed matrix [rows x K] (rows % 128 == 0, K % 64 == 0). */
+/* Bytes of one packed matrix [rows x K] (rows % 64 == 0, K % 64 == 0). */
 size_t strata_q2_matrix_bytes(int32_t rows, int32_t K);
 /* Bytes of one packed expert: 3*d*f/32*10. */
 size_t strata_moe_expert_bytes(const strata_moe_desc *desc);

@@ -55,7 +55,7 @@ def _bind(lib):
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
     lib.oracle_dequant.argtypes = [I, I, P, P, P]
-    lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, ctypes.c_long, P, P]
+    lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, ctypes.c_long, ctypes.c_long, P, P]
     lib.oracle_router_logits.argtypes = [I, I, I, P, P, P, P]
     lib.oracle_topk_softmax.argtypes = [I, I, I, P, P, P]
     lib.oracle_expert_lists.argtypes = [I, I, I, P, P, P, P]
@@ -106,25 +106,29 @@ def dequant(codes, scales_fp16):
     return W
 
 
-def unpack_q2_tiled(blob, rows: int, K: int, tile_stride: int = 2560):
-    """Codes and scales of one matrix from tiles at ``blob + t * tile_stride``."""
+def unpack_q2_tiled(blob, rows: int, K: int, panel_stride: int = None, slice_stride: int = 1280):
+    """Codes and scales of one matrix whose 64x64 tile (p, s) starts at
+    ``blob + p * panel_stride + s * slice_stride`` (a lone matrix by default)."""
     blob = _c(blob, np.uint8)
-    ntiles = rows // 128 * (K // 64)
-    assert blob.size >= (ntiles - 1) * tile_stride + 2560, "blob too small for rows x K"
+    if panel_stride is None:
+        panel_stride = (K // 64) * slice_stride
+    last = (rows // 64 - 1) * panel_stride + (K // 64 - 1) * slice_stride
+    assert blob.size >= last + 1280, "blob too small for rows x K"
     codes = np.empty((rows, K), dtype=np.uint8)
     scales = np.empty((rows, K // 32), dtype=np.uint16)
-    load().oracle_unpack_q2_tiled(rows, K, _p(blob), tile_stride, _p(codes), _p(scales))
+    load().oracle_unpack_q2_tiled(rows, K, _p(blob), panel_stride, slice_stride, _p(codes), _p(scales))
     return codes, scales.view(np.float16)
 
 
 def unpack_expert(blob, d: int, f: int) -> dict:
-    """Codes/scales of one expert from its blob section: interleaved gate/up
-    tiles (5120-byte pairs), then the down matrix (header's layout)."""
+    """Codes/scales of one expert from its blob section (header's layout):
+    gate/up tiles interleaved in (f-panel, d-slice) order, 2560-byte pairs;
+    then the down matrix [d x f] with its tiles in (f-slice, d-panel) order."""
     blob = _c(blob, np.uint8)
     gu = f * d // 64 * 20 * 2
-    gc, gs = unpack_q2_tiled(blob, f, d, 5120)
-    uc, us = unpack_q2_tiled(blob[2560:], f, d, 5120)
-    dc, ds = unpack_q2_tiled(blob[gu:], d, f, 2560)
+    gc, gs = unpack_q2_tiled(blob, f, d, (d // 64) * 2560, 2560)
+    uc, us = unpack_q2_tiled(blob[1280:], f, d, (d // 64) * 2560, 2560)
+    dc, ds = unpack_q2_tiled(blob[gu:], d, f, 1280, (d // 64) * 1280)
     return dict(gate_codes=gc, gate_scales=gs, up_codes=uc, up_scales=us, down_codes=dc, down_scales=ds)
 
 

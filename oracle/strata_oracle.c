@@ -100,22 +100,23 @@ void oracle_dequant(int rows, int K, const uint8_t *codes, const uint16_t *scale
 }
 
 /* Unpack one matrix of the tiled blob written by the library's packer, from
- * the layout the library's header documents (128-row x 64-column tiles of
- * 2560 bytes; inside a tile, row i's 64 codes occupy bytes 16i..16i+15 as four
- * little-endian 32-bit words W0..W3; column c = 16j + 8s + 2t + h of the tile
- * sits in word Wt at bit 16h + 8s + 6 - 2j; the row's two fp16 scales follow
- * at byte 2048 + 4i). Tile t starts at byte t * tile_stride (2560 for a lone matrix;
- * 5120 for the interleaved gate/up tiles of an expert). Returns one code per
- * byte and the fp16 scale bits. */
-void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long tile_stride, uint8_t *codes,
-                            uint16_t *scales)
+ * the layout the library's header documents: 64-row x 64-column tiles of
+ * 1280 bytes; inside a tile, row i's 64 codes occupy bytes 16i..16i+15 as
+ * four little-endian 32-bit words W0..W3, column c = 16j + 8s + 2t + h of the
+ * tile sitting in word Wt at bit 16h + 8s + 6 - 2j; the row's two fp16
+ * scales (columns 0-31, then 32-63) follow at byte 1024 + 4i. Tile (p, s) --
+ * rows 64p.., columns 64s.. -- starts at byte p * panel_stride +
+ * s * slice_stride (a lone matrix: slice_stride 1280, panel_stride
+ * (K/64) * 1280; an expert interleaves and reorders its tiles, see the
+ * wrapper). Returns one code per byte and the fp16 scale bits. */
+void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long panel_stride, long slice_stride,
+                            uint8_t *codes, uint16_t *scales)
 {
-    int slices = K / 64;
-    for (int p = 0; p < rows / 128; ++p)
-        for (int s = 0; s < slices; ++s) {
-            const uint8_t *tile = blob + ((size_t)p * slices + s) * (size_t)tile_stride;
-            for (int i = 0; i < 128; ++i) {
-                int r = p * 128 + i;
+    for (int p = 0; p < rows / 64; ++p)
+        for (int s = 0; s < K / 64; ++s) {
+            const uint8_t *tile = blob + (size_t)p * (size_t)panel_stride + (size_t)s * (size_t)slice_stride;
+            for (int i = 0; i < 64; ++i) {
+                int r = p * 64 + i;
                 for (int c = 0; c < 64; ++c) {
                     int j = c / 16, sh = (c / 8) % 2, t = (c % 8) / 2, h = c % 2;
                     const uint8_t *wp = tile + 16 * i + 4 * t;
@@ -125,7 +126,7 @@ void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long tile_stri
                     codes[(size_t)r * K + 64 * s + c] = (uint8_t)((w >> bit) & 3u);
                 }
                 for (int b = 0; b < 2; ++b) {
-                    const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;
+                    const uint8_t *sp = tile + 1024 + 4 * i + 2 * b;
                     scales[(size_t)r * (K / 32) + 2 * s + b] = (uint16_t)(sp[0] | (sp[1] << 8));
                 }
             }

@@ -44,7 +44,7 @@ def bf16_rne_exact(v: float) -> int:
 
 
 def load_tile_example():
-    blob = np.zeros(2560, dtype=np.uint8)
+    blob = np.zeros(1280, dtype=np.uint8)
     expects = []
     with open(os.path.join(GOLD, "q2_tile_example.txt")) as fh:
         for line in fh:
@@ -141,13 +141,13 @@ def check_bf16_convert():
 
 def check_tile_example():
     blob, expects = load_tile_example()
-    codes, scales = O.unpack_q2_tiled(blob, 128, 64)
+    codes, scales = O.unpack_q2_tiled(blob, 64, 64)
     W = O.dequant(codes, scales)
     for r, c, code, val in expects:
         assert codes[r, c] == code, f"code at ({r},{c}) = {codes[r, c]}, expected {code}"
         assert W[r, c] == val, f"weight at ({r},{c}) = {W[r, c]}, expected {val}"
-    # rows 2..126 are all code 0 with scale 1 -> -1.5 everywhere
-    assert np.all(W[2:127] == -1.5)
+    # rows 2..62 are all code 0 with scale 1 -> -1.5 everywhere
+    assert np.all(W[2:63] == -1.5)
 
 
 def check_dequant_rules():

@@ -25,7 +25,7 @@ MUTANTS = [
      "for (int j = 0; j < k; ++j)\n            for (int t = 0; t < T; ++t)\n                if (idx[(size_t)t * k + j] == e) {"),
     ("unpack_bit", "int bit = 16 * h + 8 * sh + 6 - 2 * j;", "int bit = 16 * h + 8 * sh + 2 * j;"),
     ("unpack_word", "const uint8_t *wp = tile + 16 * i + 4 * t;", "const uint8_t *wp = tile + 16 * i + 4 * j;"),
-    ("unpack_scale_order", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * (1 - b);"),
+    ("unpack_scale_order", "const uint8_t *sp = tile + 1024 + 4 * i + 2 * b;", "const uint8_t *sp = tile + 1024 + 4 * i + 2 * (1 - b);"),
     ("rms_no_mean", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
     ("rms_eps_outside", "double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss / d) + eps;"),
     ("bf16_truncate", "double r = nearbyint(v / q) * q;", "double r = trunc(v / q) * q;"),
