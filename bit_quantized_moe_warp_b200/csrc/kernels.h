@@ -69,8 +69,10 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
 // --- prefill experts (tensor cores)
 void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
                          const Shape &s, int num_sms, cudaStream_t st);
+// writes w * W_down h per pair into ws.xp (fp16 [pairs x d]); launch_combine sums them into y
 void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
                          const Shape &s, int num_sms, cudaStream_t st);
+void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const Shape &s, cudaStream_t st);
 
 // --- misc
 void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cudaStream_t st);

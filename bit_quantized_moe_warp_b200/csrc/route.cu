@@ -166,31 +166,28 @@ __device__ void warp_topk(const float *__restrict__ lrow, int E, int k, int *sel
 }
 
 // ------------------------------------------------------------ large lists
-// Prefill sizes. (1) top-k per token, per-256-token-block expert counts.
+// Prefill sizes. (1) top-k per token, one warp per token; expert counts per
+// 256-token block accumulated with atomics (blk_counts zeroed beforehand).
+constexpr int kTopkTokensPerCta = 32;
 __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E, int k) {
-    __shared__ int s_cnt[1024];
     __shared__ int s_idx[8][32];
     __shared__ float s_w[8][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int e = threadIdx.x; e < E; e += 256) s_cnt[e] = 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) ws.meta[META_N_TOKENS] = T;
-    __syncthreads();
-    const int t0 = blockIdx.x * kRouteBlock;
-    for (int i = warp; i < kRouteBlock; i += 8) {
-        int t = t0 + i;
+    const int t0 = blockIdx.x * kTopkTokensPerCta;
+    for (int i = warp; i < kTopkTokensPerCta; i += 8) {
+        const int t = t0 + i;
         if (t >= T) break;
         warp_topk(ws.logits + (size_t)t * E, E, k, s_idx[warp], s_w[warp]);
         __syncwarp();
         if (lane < k) {
-            int e = s_idx[warp][lane];
+            const int e = s_idx[warp][lane];
             ws.topk_idx[(size_t)t * k + lane] = e;
             ws.topk_w[(size_t)t * k + lane] = s_w[warp][lane];
-            atomicAdd(&s_cnt[e], 1);
+            atomicAdd(&ws.blk_counts[(size_t)(t / kRouteBlock) * E + e], 1);
         }
         __syncwarp();
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += 256) ws.blk_counts[(size_t)blockIdx.x * E + e] = s_cnt[e];
 }
 
 // (2) one block: expert totals, offsets, per-block bases (in place in
@@ -328,7 +325,8 @@ void launch_router_gemm(const void *x, const float *W, const float *bias, float 
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
                         cudaStream_t st) {
     const int nblk = (T + kRouteBlock - 1) / kRouteBlock;
-    k_topk_blocks<<<nblk, 256, 0, st>>>(ws, T, s.E, s.k);
+    cudaMemsetAsync(ws.blk_counts, 0, (size_t)nblk * s.E * sizeof(int32_t), st);
+    k_topk_blocks<<<(T + kTopkTokensPerCta - 1) / kTopkTokensPerCta, 256, 0, st>>>(ws, T, s.E, s.k);
     k_lists_scan<<<1, 1024, 0, st>>>(ws, T, s.E, max_tiles1, max_tiles2);
     k_lists_scatter<<<nblk, 256, (size_t)s.E * 8 * sizeof(uint32_t), st>>>(ws, T, s.E, s.k);
 }

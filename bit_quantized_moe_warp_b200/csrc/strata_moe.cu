@@ -395,12 +395,12 @@ static strata_status route_impl(strata_moe_layer L, const void *x, const float *
 static strata_status experts_impl(strata_moe_layer L, const void *x, const void *blob, float *y, int T, bool acc,
                                   cudaStream_t st) {
     const uint8_t *b = static_cast<const uint8_t *>(blob);
-    if (!acc) CUDA_TRY(cudaMemsetAsync(y, 0, (size_t)T * L->shape.d * sizeof(float), st));
     launch_gather_xp(L->ws, x, T, L->shape, st);
     stage_mark(L, 2, st);
     launch_expert_gemm1(L->ws, b, L->maps1, L->plan.max_tiles1, L->shape, L->num_sms, st);
     stage_mark(L, 3, st);
     launch_expert_gemm2(L->ws, b, y, L->maps2, L->plan.max_tiles2, L->shape, L->num_sms, st);
+    launch_combine(L->ws, y, acc, T, L->shape, st);  // y = (or +=) the sum of each token's k expert outputs
     return check_launch("expert kernels");
 }
 
