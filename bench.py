@@ -31,6 +31,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s (decode & 8K prefill) + % of HBM / tensor roofline"
+
+# DRAM bytes (read + write) of one launch of each workload's dominant kernel
+# from one ncu capture (profiles/*.md gives the command). Set to None when the
+# kernel changes after the capture.
+MEASURED_TRAFFIC = {
+    "decode": 19056896,             # k_decode_fused<1>, profiles/decode_fused_T1.md
+    "prefill": 557109504 + 126158592,  # k_expert_gemm<0>, profiles/prefill_expert_gemm_8192.md
+}
 PREFILL_KERNELS = 8
 
 
@@ -323,14 +331,15 @@ def roofline(w, dom, hbm, tf_burst, peak_src):
         bytes_ = decode_bytes(w, dom["n_active"])
         ach = bytes_ / (dom["dom_ms"] * 1e-3) / 1e9
         return {"bound": "hbm", "kernel": "k_decode_fused (whole layer, one launch)", "achieved": ach, "peak": hbm,
-                "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                "unit": "GB/s", "frac": ach / hbm, "traffic": MEASURED_TRAFFIC.get(w.name),
                 "algorithmic_bytes_per_launch": bytes_, "selected_experts_per_launch": dom["n_active"],
                 "avg_launch_ms": dom["dom_ms"], "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
                 "layer_call_ms": dom["step_ms"]}
     flops = dom["T"] * w.k * 2 * 2 * w.d * w.f
     ach = flops / (dom["dom_ms"] * 1e-3) / 1e12
     return {"bound": "tensor", "kernel": "k_expert_gemm<0> (gate/up + SwiGLU)", "achieved": ach, "peak": tf_burst,
-            "unit": "TFLOP/s", "frac": ach / tf_burst, "traffic": None, "algorithmic_flops_per_launch": flops,
+            "unit": "TFLOP/s", "frac": ach / tf_burst, "traffic": MEASURED_TRAFFIC.get(w.name),
+            "algorithmic_flops_per_launch": flops,
             "avg_launch_ms": dom["dom_ms"], "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops; fp16 same rate)",
             "layer_call_ms": dom["step_ms"],
             "layer_expert_TFLOPs": dom["T"] * w.k * 6 * w.d * w.f / (dom["step_ms"] * 1e-3) / 1e12}
