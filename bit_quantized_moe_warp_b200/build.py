@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libstrata_moe.so")
-SOURCES = ["strata_moe.cu", "route.cu", "decode_fused.cu", "prefill_gemm.cu", "misc.cu", "route_noalloc.cu"]
+SOURCES = ["strata_moe.cu", "route.cu", "decode_fused.cu", "prefill_gemm.cu", "misc.cu", "route_noalloc.cu", "router_gemm.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]

@@ -30,6 +30,7 @@ struct Workspace {
     int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
     int4 *tiles2;         // down GEMM tiles
     void *xn;             // bf16 [T * d]         stack: normalised input
+    void *w_hi, *w_lo;    // bf16 [E * d] each    prefill router: bf16 split of W_r
     uint32_t *sync;       // [2]     fused decode: grid barrier, exit count
 };
 
@@ -49,11 +50,19 @@ struct TmaMaps {
     CUtensorMap m[5];  // box rows 16, 32, 64, 128, 256
 };
 
+// prefill router on the tensor cores: W_hi / W_lo [E x d] (boxes 64 x 128),
+// x [T x d] (box 64 x 256), bf16, 128-byte swizzle
+struct RouterMaps {
+    CUtensorMap w_hi, w_lo, x;
+};
+
 // --- routing
 void launch_router_gemv(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
                         cudaStream_t st);
-void launch_router_gemm(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
-                        cudaStream_t st);
+// prefill sizes: splits W into bf16 hi/lo (ws.w_hi, ws.w_lo), then the tensor-core GEMM
+void launch_router_tc(const Workspace &ws, const RouterMaps &maps, const float *W, const float *bias, float *logits,
+                      int T, const Shape &s, int num_sms, cudaStream_t st);
+cudaError_t init_router_attributes(int max_smem);
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
                         cudaStream_t st);
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st);

@@ -13,8 +13,8 @@
 //     of gate and up, two accumulators G, U [128 x N] share the token
 //     operand; the epilogue writes H = silu(G) * U (fp16, pair-major).
 //   MODE 1 (down): per tile of <= 256 pairs and 128-row panel of down,
-//     O = W_down H^T; the epilogue stores w * O (fp16, pair-major) and a
-//     combine kernel sums each token's k rows into y (no atomics).
+//     O = W_down H^T; the epilogue stores O (fp16, pair-major) and a
+//     combine kernel sums each token's k rows, weighted, into y (no atomics).
 //
 // Warp roles (448 threads): warp 0 issues the copies, warp 1 issues the MMAs
 // (one thread), warps 2-5 drain the accumulators, warps 6-13 dequantise.
@@ -64,8 +64,7 @@ struct GemmArgs {
     const int4 *tiles;
     const int *n_tiles;
     __half *H;         // MODE 0 output
-    __half *O;         // MODE 1 output: w * W_down h per pair [pairs x d]
-    const float *pair_w;
+    __half *O;         // MODE 1 output: W_down h per pair [pairs x d]
     uint32_t *status;
 };
 
@@ -213,10 +212,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        if (c0 + i < n) {
-                            const int pr = p0 + c0 + i;
-                            a.O[(size_t)pr * a.ldo + feat] = __float2half_rn(a.pair_w[pr] * o[i]);
-                        }
+                        if (c0 + i < n) a.O[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(o[i]);
                 }
             }
             tc_fence_before();
@@ -316,11 +312,13 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
     launch_gemm<0>(maps, a, num_sms, st);
 }
 
-// y[t] (+)= sum_j O[pair_of(t, j)]: one CTA per token, 8 features per thread.
+// y[t] (+)= sum_j w_j O[pair_of(t, j)]: one CTA per token, 8 features per thread.
 __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, const int *__restrict__ pair_of,
-                                                 float *__restrict__ y, int d, int k, int accumulate) {
+                                                 const float *__restrict__ topk_w, float *__restrict__ y, int d,
+                                                 int k, int accumulate) {
     const int t = blockIdx.x;
     const int *po = pair_of + (size_t)t * k;
+    const float *wt = topk_w + (size_t)t * k;
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
         float acc[8];
 #pragma unroll
@@ -328,11 +326,12 @@ __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, c
         for (int j = 0; j < k; ++j) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(O + (size_t)po[j] * d + c));
             const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+            const float w = wt[j];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float2 f = __half22float2(h[q]);
-                acc[2 * q] += f.x;
-                acc[2 * q + 1] += f.y;
+                acc[2 * q] = fmaf(w, f.x, acc[2 * q]);
+                acc[2 * q + 1] = fmaf(w, f.y, acc[2 * q + 1]);
             }
         }
         float4 *yr = reinterpret_cast<float4 *>(y + (size_t)t * d + c);
@@ -348,7 +347,8 @@ __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, c
 
 void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const Shape &s, cudaStream_t st) {
     if (T <= 0) return;
-    k_combine<<<T, 256, 0, st>>>(static_cast<const __half *>(ws.xp), ws.pair_of, y, s.d, s.k, accumulate ? 1 : 0);
+    k_combine<<<T, 256, 0, st>>>(static_cast<const __half *>(ws.xp), ws.pair_of, ws.topk_w, y, s.d, s.k,
+                                 accumulate ? 1 : 0);
 }
 
 void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
@@ -366,7 +366,6 @@ void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, con
     a.n_tiles = ws.meta + META_N_TILES2;
     (void)y;
     a.O = static_cast<__half *>(ws.xp);  // the gathered inputs are dead once gate/up has run
-    a.pair_w = ws.pair_w;
     a.status = ws.status;
     (void)max_tiles;
     launch_gemm<1>(maps, a, num_sms, st);

@@ -49,54 +49,6 @@ __global__ void __launch_bounds__(128) k_router_gemv(const __nv_bfloat16 *__rest
     }
 }
 
-// ------------------------------------------------------------ router GEMM
-// Prefill sizes: tiled fp32 SIMT GEMM, logits[T x E] = X W_r^T + b.
-// 64 tokens x 64 experts per block, 16-wide K steps, 4x4 outputs per thread,
-// K summed in ascending order per output.
-__global__ void __launch_bounds__(256) k_router_gemm(const __nv_bfloat16 *__restrict__ x,
-                                                      const float *__restrict__ W,
-                                                      const float *__restrict__ bias, float *__restrict__ logits,
-                                                      int T, int d, int E) {
-    __shared__ float xs[16][64 + 4];
-    __shared__ float wsm[16][64 + 4];
-    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < d; k0 += 16) {
-        // 64 rows x 16 k of x and of W: 1024 elements each, 4 per thread
-        for (int i = threadIdx.x; i < 1024; i += 256) {
-            int r = i >> 4, kk = i & 15;
-            int t = t0 + r, e = e0 + r;
-            xs[kk][r] = (t < T) ? __bfloat162float(x[(size_t)t * d + k0 + kk]) : 0.f;
-            wsm[kk][r] = (e < E) ? W[(size_t)e * d + k0 + kk] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-            float a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = wsm[kk][tx * 4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int t = t0 + ty * 4 + i;
-        if (t >= T) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int e = e0 + tx * 4 + j;
-            if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
-        }
-    }
-}
-
 // ------------------------------------------------------------ top-k
 // One warp per token: lane l owns experts l, l+32, ... (E <= 1024). k rounds
 // of a warp arg-max over (logit descending, index ascending); only the
@@ -314,12 +266,6 @@ void launch_router_gemv(const void *x, const float *W, const float *bias, float 
         k_router_gemv<4><<<grid, block, 0, st>>>(xb, W, bias, logits, T, s.d, s.E);
     else
         k_router_gemv<16><<<grid, block, 0, st>>>(xb, W, bias, logits, T, s.d, s.E);
-}
-
-void launch_router_gemm(const void *x, const float *W, const float *bias, float *logits, int T, const Shape &s,
-                        cudaStream_t st) {
-    dim3 grid((s.E + 63) / 64, (T + 63) / 64), block(256);
-    k_router_gemm<<<grid, block, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), W, bias, logits, T, s.d, s.E);
 }
 
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,

@@ -102,7 +102,7 @@ static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
-    size_t off[20];
+    size_t off[22];
     size_t total;
     int max_tiles1, max_tiles2;
 };
@@ -115,7 +115,7 @@ static Plan plan_workspace(const strata_moe_desc *d) {
     Plan p{};
     p.max_tiles1 = (int)((P + kGemm1N - 1) / kGemm1N + E);
     p.max_tiles2 = (int)((P + kGemm2N - 1) / kGemm2N + E);
-    const size_t sz[20] = {
+    const size_t sz[22] = {
         256,                                      // 0 status
         64 * 4,                                   // 1 meta
         T * E * 4,                                // 2 logits
@@ -136,9 +136,11 @@ static Plan plan_workspace(const strata_moe_desc *d) {
         (size_t)p.max_tiles2 * 16,                // 17 tiles2
         T * (size_t)s.d * 2,                      // 18 xn
         (2 + E) * 4,                              // 19 sync
+        E * (size_t)s.d * 2,                      // 20 w_hi
+        E * (size_t)s.d * 2,                      // 21 w_lo
     };
     size_t o = 0;
-    for (int i = 0; i < 20; ++i) {
+    for (int i = 0; i < 22; ++i) {
         p.off[i] = o;
         o += (sz[i] + 255) & ~(size_t)255;
     }
@@ -168,6 +170,8 @@ static Workspace carve(uint8_t *base, const Plan &p) {
     w.tiles2 = reinterpret_cast<int4 *>(base + p.off[17]);
     w.xn = base + p.off[18];
     w.sync = reinterpret_cast<uint32_t *>(base + p.off[19]);
+    w.w_hi = base + p.off[20];
+    w.w_lo = base + p.off[21];
     return w;
 }
 
@@ -207,12 +211,29 @@ static strata_status make_maps(TmaMaps &m, void *base, size_t rows, int K) {
     return STRATA_OK;
 }
 
+// Map over a row-major bf16 matrix [rows x K] with boxes of 64 columns x
+// box_rows rows and 128-byte swizzle; rows beyond the matrix read as zeros.
+static strata_status make_bf16_map(CUtensorMap *m, const void *base, size_t rows, int K, int box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return fail(STRATA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(STRATA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return STRATA_OK;
+}
+
 namespace strata {
 cudaError_t init_gemm_attributes(int max_smem);
 static cudaError_t init_kernel_attributes(int device, const Shape &s, int max_tokens, int num_sms) {
     int max_smem = 0;
     cudaError_t e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     if (e == cudaSuccess) e = init_gemm_attributes(max_smem);
+    if (e == cudaSuccess) e = init_router_attributes(max_smem);
     if (e == cudaSuccess) e = init_fused_attributes(s, max_tokens, max_smem, num_sms);
     return e;
 }
@@ -235,6 +256,7 @@ struct strata_moe_layer_s {
     Plan plan;
     Workspace ws;
     TmaMaps maps1, maps2;
+    RouterMaps rmaps;  // W_hi / W_lo fixed at creation; x encoded per call
     bool fused_ok;   // the one-launch streaming layer fits this shape
     int max_smem;
     StackGraph graph;
@@ -331,7 +353,9 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
     }
     const size_t P = (size_t)desc->max_tokens * desc->top_k;
     if ((s = make_maps(L->maps1, L->ws.xp, P, L->shape.d)) != STRATA_OK ||
-        (s = make_maps(L->maps2, L->ws.hbuf, P, L->shape.f)) != STRATA_OK) {
+        (s = make_maps(L->maps2, L->ws.hbuf, P, L->shape.f)) != STRATA_OK ||
+        (s = make_bf16_map(&L->rmaps.w_hi, L->ws.w_hi, L->shape.E, L->shape.d, 128)) != STRATA_OK ||
+        (s = make_bf16_map(&L->rmaps.w_lo, L->ws.w_lo, L->shape.E, L->shape.d, 128)) != STRATA_OK) {
         if (L->owns_ws) cudaFree(L->ws_mem);
         delete L;
         return s;
@@ -382,12 +406,25 @@ static bool use_decode(strata_moe_layer L, int T) {
     return T <= kDecMaxT && L->fused_ok && !(L->desc.flags & STRATA_FORCE_PREFILL);
 }
 
+// logits of T tokens: GEMV for decode sizes, the tensor-core GEMM (bf16
+// split of W) beyond
+static strata_status router_impl(strata_moe_layer L, const void *x, const float *W, const float *bias, float *logits,
+                                 int T, cudaStream_t st) {
+    if (T <= kDecMaxT) {
+        launch_router_gemv(x, W, bias, logits, T, L->shape, st);
+        return STRATA_OK;
+    }
+    RouterMaps maps = L->rmaps;
+    strata_status s = make_bf16_map(&maps.x, x, (size_t)T, L->shape.d, 256);
+    if (s != STRATA_OK) return s;
+    launch_router_tc(L->ws, maps, W, bias, logits, T, L->shape, L->num_sms, st);
+    return STRATA_OK;
+}
+
 static strata_status route_impl(strata_moe_layer L, const void *x, const float *W, const float *bias, int T,
                                 cudaStream_t st) {
-    if (T <= kDecMaxT)
-        launch_router_gemv(x, W, bias, L->ws.logits, T, L->shape, st);
-    else
-        launch_router_gemm(x, W, bias, L->ws.logits, T, L->shape, st);
+    strata_status s = router_impl(L, x, W, bias, L->ws.logits, T, st);
+    if (s != STRATA_OK) return s;
     launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st);
     return check_launch("routing kernels");
 }
@@ -444,10 +481,7 @@ extern "C" strata_status strata_moe_router_logits(strata_moe_layer L, const void
         return fail(STRATA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
     if (T == 0) return STRATA_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (T <= kDecMaxT)
-        launch_router_gemv(x, W, L->desc.router_bias, logits, T, L->shape, st);
-    else
-        launch_router_gemm(x, W, L->desc.router_bias, logits, T, L->shape, st);
+    if ((s = router_impl(L, x, W, L->desc.router_bias, logits, T, st)) != STRATA_OK) return s;
     return check_launch("router kernel");
 }
 
