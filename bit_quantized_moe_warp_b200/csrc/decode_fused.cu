@@ -248,18 +248,29 @@ STRATA_DEV void tile_mma(const TileRows &w, BSrc bsrc, ZSrc zsrc, float (&out)[N
 // one warp: z[b] = sum over the block's columns k of (base_j(k) + 1.5) x_k,
 // i.e. sum_j base_j X_j + 1.5 X_b. Lane l reads columns 2l, 2l+1 of each
 // tile (step j = l / 8, block l / 16) and the 16 lanes of a block reduce by
-// shuffles, so the reads are conflict-free.
+// shuffles, so the reads are conflict-free; four tiles at a time keep four
+// independent shuffle chains in flight.
 STRATA_DEV void row_block_constants(const __half *row, int ncols, float *z) {
     const int lane = threadIdx.x & 31;
     const float wgt = step_base(lane >> 3) + 1.5f;
-    for (int c0 = 0; c0 < ncols; c0 += 64) {
-        const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(row + c0 + 2 * lane));
-        float sum = wgt * (v.x + v.y);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 8);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        if ((lane & 15) == 0) z[c0 / 32 + (lane >> 4)] = sum;
+    for (int c0 = 0; c0 < ncols; c0 += 256) {
+        float sum[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            sum[q] = 0.f;
+            if (c0 + 64 * q < ncols) {
+                const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(row + c0 + 64 * q + 2 * lane));
+                sum[q] = wgt * (v.x + v.y);
+            }
+        }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sum[q] += __shfl_xor_sync(0xffffffffu, sum[q], o);
+        if ((lane & 15) == 0)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (c0 + 64 * q < ncols) z[(c0 + 64 * q) / 32 + (lane >> 4)] = sum[q];
     }
 }
 
@@ -501,8 +512,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         for (int c = tid; c < d / 2; c += 512)  // zero row (empty MMA token slots)
             reinterpret_cast<uint32_t *>(xh + (size_t)T * dpx)[c] = 0u;
         compute_sync();
-        for (int r = warp; r <= T; r += kFusedComputeWarps)  // per-block constants of x (and the zero row)
-            row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
+        for (int i = tid; i < d / 32; i += 512) xz[(size_t)T * (d / 32) + i] = 0.f;  // the zero row's constants
         // router: warp -> (row, quarter of K); each lane keeps 16 K-values of
         // W in registers per 512-column step and walks the tokens
         if (wstaged) mbar_wait(&wbar, 0, status, &s_abort);
@@ -570,7 +580,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             for (int j = lane; j < k; j += 32) ex += expf(sel_val[warp * k + j] - vmax);
             const float den = warp_sum(ex);
             for (int j = lane; j < k; j += 32) sel_w[warp * k + j] = expf(sel_val[warp * k + j] - vmax) / den;
+        } else {  // warps without a token meanwhile compute the per-block constants of x (used in phase 2)
+            for (int r = warp - T; r < T; r += kFusedComputeWarps - T)
+                row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         }
+        if (T >= kFusedComputeWarps)  // no warp was free
+            for (int r = warp; r < T; r += kFusedComputeWarps)
+                row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         compute_sync();
         for (int i = tid; i < T * k; i += 512) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
         compute_sync();
