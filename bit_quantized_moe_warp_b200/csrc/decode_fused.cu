@@ -514,7 +514,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         compute_sync();
         for (int i = tid; i < d / 32; i += 512) xz[(size_t)T * (d / 32) + i] = 0.f;  // the zero row's constants
         // router: warp -> (row, quarter of K); each lane keeps 16 K-values of
-        // W in registers per 512-column step and walks the tokens
+        // W in registers per 512-column step and accumulates every token;
+        // the tokens' warp sums run interleaved at the end
         if (wstaged) mbar_wait(&wbar, 0, status, &s_abort);
         const int q4 = d / 4;
         for (int u = warp; u < nr * 4 && !s_abort; u += kFusedComputeWarps) {
@@ -522,35 +523,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             const float *wrow = wstaged ? reinterpret_cast<const float *>(bufs + woff) + (size_t)rr * d
                                         : a.W + (size_t)(r0 + rr) * d;
             const int cbase = kq * q4;
+            float acc[TT];
+#pragma unroll
+            for (int t = 0; t < TT; ++t) acc[t] = 0.f;
             for (int c0 = 0; c0 < q4; c0 += 512) {
                 const int ncol = min(512, q4 - c0);  // a multiple of 32 (d is a multiple of 128)
-                float4 wv[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    wv[i] = 128 * i + 4 * lane < ncol
-                                ? *reinterpret_cast<const float4 *>(wrow + cbase + c0 + 128 * i + 4 * lane)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int t = 0; t < T; ++t) {
-                    const __half *xr = xh + (size_t)t * dpx + cbase + c0;
-                    float acc = 0.f;
+                for (int i = 0; i < 4; ++i) {
+                    if (128 * i + 4 * lane < ncol) {
+                        const float4 wv = *reinterpret_cast<const float4 *>(wrow + cbase + c0 + 128 * i + 4 * lane);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (128 * i + 4 * lane < ncol) {
-                            const __half2 *xp = reinterpret_cast<const __half2 *>(xr + 128 * i + 4 * lane);
-                            const float2 x01 = __half22float2(xp[0]), x23 = __half22float2(xp[1]);
-                            acc = fmaf(wv[i].x, x01.x, acc);
-                            acc = fmaf(wv[i].y, x01.y, acc);
-                            acc = fmaf(wv[i].z, x23.x, acc);
-                            acc = fmaf(wv[i].w, x23.y, acc);
+                        for (int t = 0; t < TT; ++t) {
+                            if (t < T) {
+                                const uint2 xv =
+                                    *reinterpret_cast<const uint2 *>(xh + (size_t)t * dpx + cbase + c0 + 128 * i + 4 * lane);
+                                const float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.x));
+                                const float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.y));
+                                acc[t] = fmaf(wv.x, x01.x, acc[t]);
+                                acc[t] = fmaf(wv.y, x01.y, acc[t]);
+                                acc[t] = fmaf(wv.z, x23.x, acc[t]);
+                                acc[t] = fmaf(wv.w, x23.y, acc[t]);
+                            }
                         }
-                    }
-                    acc = warp_sum(acc);
-                    if (lane == 0) {
-                        float *dst = lsm + ((size_t)t * kRouterRowsMax + rr) * 4 + kq;
-                        *dst = (c0 == 0) ? acc : *dst + acc;
                     }
                 }
             }
+#pragma unroll
+            for (int t = 0; t < TT; ++t) acc[t] = warp_sum(acc[t]);
+            if (lane == 0)
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    if (t < T) lsm[((size_t)t * kRouterRowsMax + rr) * 4 + kq] = acc[t];
         }
         if (tid < nr) cp_async_wait_all();
         compute_sync();
