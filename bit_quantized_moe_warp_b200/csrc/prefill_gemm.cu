@@ -225,8 +225,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
         const int row = dt & 127, sub = dt >> 7;
         const int mat = (MODE == 0) ? sub : 0;
         const int c_lo = (MODE == 0) ? 0 : 4 * sub, c_hi = (MODE == 0) ? 8 : 4 * sub + 4;
-        const __half2 k1027 = __floats2half2_rn(1027.f, 1027.f);
-        const __half2 khalf = __floats2half2_rn(0.5f, 0.5f);
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -242,25 +240,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                 const int ri = row & 63;
                 const uint4 cw = *reinterpret_cast<const uint4 *>(wt + 16 * ri);
                 uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + kTileScaleOffset + 4 * ri);
-                const __half2 s01 = __hmul2(*reinterpret_cast<__half2 *>(&scb), khalf);  // (s0/2, s1/2)
+                const __half2 s01 = *reinterpret_cast<__half2 *>(&scb);
                 const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                const uint32_t words8[4] = {cw.x >> 8, cw.y >> 8, cw.z >> 8, cw.w >> 8};
                 uint8_t *arow = A_at(st, mat) + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {  // output chunk c: columns 8c .. 8c+7
                     if (c < c_lo || c >= c_hi) continue;
                     const __half2 sc = (c < 4) ? sh0 : sh1;
-                    // columns 8c + 2t, 8c + 2t + 1 sit in word t, halves 0/1, at bit
-                    // 8 (c & 1) + 6 - 2 (c >> 1); bring them to bits 1-2 of each half
-                    const int pos = 8 * (c & 1) + 6 - 2 * (c >> 1);
+                    // Columns 8c + 2t, 8c + 2t + 1 (step j = c / 2, half s = c % 2)
+                    // sit in word t at bits 8s + 6 - 2j and 16 + 8s + 6 - 2j. With
+                    // the exponent that gives bit 6 - 2j the place value 1, the
+                    // masked pair reads as the exact fp16 values base_j + code
+                    // (base 16, 64, 256, 1024); subtracting base_j + 1.5 is exact
+                    // for j < 3 (17.5, 65.5, 257.5), and in two exact steps for
+                    // j = 3; one multiply by the scale rounds once.
+                    const int j = c >> 1;
+                    const uint32_t m = 0x00030003u << (6 - 2 * j);
+                    const uint32_t g = j == 0 ? 0x4C004C00u : j == 1 ? 0x54005400u : j == 2 ? 0x5C005C00u : 0x64006400u;
                     uint32_t out[4];
 #pragma unroll
                     for (int pr = 0; pr < 4; ++pr) {
-                        const uint32_t w = words[pr];
-                        uint32_t v = (pos == 0) ? (w << 1) : (w >> (pos - 1));
-                        v = (v & 0x00060006u) | 0x64006400u;  // fp16 1024 + 2c in both halves
+                        uint32_t v = (((c & 1) ? words8[pr] : words[pr]) & m) | g;
                         __half2 h = *reinterpret_cast<__half2 *>(&v);
-                        h = __hmul2(__hsub2(h, k1027), sc);    // (2c - 3) * s/2 = (c - 1.5) s
+                        if (j < 3) {
+                            const float off = j == 0 ? 17.5f : j == 1 ? 65.5f : 257.5f;
+                            h = __hsub2(h, __floats2half2_rn(off, off));
+                        } else {
+                            h = __hsub2(__hsub2(h, __floats2half2_rn(1024.f, 1024.f)), __floats2half2_rn(1.5f, 1.5f));
+                        }
+                        h = __hmul2(h, sc);  // (c - 1.5) s
                         out[pr] = *reinterpret_cast<uint32_t *>(&h);
                     }
                     *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
