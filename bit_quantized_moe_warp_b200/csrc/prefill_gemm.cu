@@ -30,7 +30,7 @@ template <int MODE>
 struct GCfg;
 template <>
 struct GCfg<0> {
-    static constexpr int NMAT = 2, NMAX = kGemm1N, STAGES = 3;
+    static constexpr int NMAT = 2, NMAX = kGemm1N, STAGES = 4;
 };
 template <>
 struct GCfg<1> {

@@ -120,7 +120,7 @@ __device__ void warp_topk(const float *__restrict__ lrow, int E, int k, int *sel
 // ------------------------------------------------------------ large lists
 // Prefill sizes. (1) top-k per token, one warp per token; expert counts per
 // 256-token block accumulated with atomics (blk_counts zeroed beforehand).
-constexpr int kTopkTokensPerCta = 32;
+constexpr int kTopkTokensPerCta = 8;  // one token per warp
 __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E, int k) {
     __shared__ int s_idx[8][32];
     __shared__ float s_w[8][32];
@@ -160,28 +160,60 @@ __global__ void __launch_bounds__(1024) k_lists_scan(Workspace ws, int T, int E,
         }
         s_tot[e] = tot;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0, f1 = 0, p1 = 0, f2 = 0, p2 = 0;
-        for (int i = 0; i < E; ++i) {
-            s_off[i] = run;
-            run += s_tot[i];
-            s_f1[i] = f1;
-            f1 += s_tot[i] / kGemm1N;
-            s_p1[i] = p1;
-            p1 += (s_tot[i] % kGemm1N) != 0;
-            s_f2[i] = f2;
-            f2 += s_tot[i] / kGemm2N;
-            s_p2[i] = p2;
-            p2 += (s_tot[i] % kGemm2N) != 0;
+    // exclusive scans over the experts of: the pair count, the full and the
+    // partial gate/up tiles, the full and the partial down tiles (a block
+    // scan: warp shuffles, then the warp totals)
+    __shared__ int s_wsum[32][5];
+    {
+        const int t = e < E ? tot : 0;
+        int v[5] = {t, t / kGemm1N, (t % kGemm1N) != 0, t / kGemm2N, (t % kGemm2N) != 0};
+        int incl[5];
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+        for (int q = 0; q < 5; ++q) incl[q] = v[q];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+            for (int q = 0; q < 5; ++q) {
+                const int u = __shfl_up_sync(0xffffffffu, incl[q], o);
+                if (lane >= o) incl[q] += u;
+            }
+        if (lane == 31)
+#pragma unroll
+            for (int q = 0; q < 5; ++q) s_wsum[warp][q] = incl[q];
+        __syncthreads();
+        if (warp == 0) {
+#pragma unroll
+            for (int q = 0; q < 5; ++q) {
+                int w = s_wsum[lane][q];  // 32 warps of 32 threads cover 1024 experts
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, w, o);
+                    if (lane >= o) w += u;
+                }
+                s_wsum[lane][q] = w;  // inclusive over warps
+            }
         }
-        s_off[E] = run;
-        s_f1[E] = f1;
-        s_p1[E] = p1;
-        s_f2[E] = f2;
-        s_p2[E] = p2;
-        ws.meta[META_N_TILES1] = min(f1 + p1, max_tiles1);
-        ws.meta[META_N_TILES2] = min(f2 + p2, max_tiles2);
+        __syncthreads();
+        int ex[5];
+#pragma unroll
+        for (int q = 0; q < 5; ++q) ex[q] = (warp ? s_wsum[warp - 1][q] : 0) + incl[q] - v[q];
+        if (e < E) {
+            s_off[e] = ex[0];
+            s_f1[e] = ex[1];
+            s_p1[e] = ex[2];
+            s_f2[e] = ex[3];
+            s_p2[e] = ex[4];
+        }
+        if (threadIdx.x == 0) {
+            s_off[E] = s_wsum[31][0];
+            s_f1[E] = s_wsum[31][1];
+            s_p1[E] = s_wsum[31][2];
+            s_f2[E] = s_wsum[31][3];
+            s_p2[E] = s_wsum[31][4];
+            ws.meta[META_N_TILES1] = min(s_wsum[31][1] + s_wsum[31][2], max_tiles1);
+            ws.meta[META_N_TILES2] = min(s_wsum[31][3] + s_wsum[31][4], max_tiles2);
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) ws.offsets[E] = s_off[E];
