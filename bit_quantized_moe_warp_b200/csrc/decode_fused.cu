@@ -47,6 +47,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace strata {
 
@@ -121,16 +122,6 @@ __host__ __device__ inline FusedSmem fused_plan(int T, int TT, int d, int E, int
     p.bufs = o;    o += (size_t)nbuf * kChunkBytes;
     p.total = o;
     return p;
-}
-
-// monotone map of a float to uint32 (+0 and -0 both map to 0x80000000);
-// every finite or infinite value maps above 0, the "taken" marker
-STRATA_DEV uint32_t ordered_key(float v) {
-    uint32_t u = __float_as_uint(v + 0.0f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-STRATA_DEV float key_value(uint32_t key) {
-    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // time-bounded spin until *ctr >= target (acquire); false on timeout/abort
@@ -325,69 +316,6 @@ STRATA_DEV void down_rows(const TileRows &w, const uint32_t (&bf)[NT][4][2], con
             zb = zf[n][blk][1];
         },
         reinterpret_cast<float(&)[NTA][4]>(o));
-}
-
-// ------------------------------------------------------------ top-k
-// One warp, one token. Lane l holds the logits of experts KPL*l ..
-// KPL*l + KPL - 1 as ordered keys, sorted in registers (bitonic network,
-// key descending, then expert ascending). Among equal keys the lowest lane
-// holds the lowest expert index, so each of the k rounds takes the warp max
-// of the lanes' heads and the lowest lane holding it (ballot), which pops
-// its head.
-template <int KPL>
-STRATA_DEV void token_topk(const float *logits, int t, int E, int k, int *sel_idx, float *sel_val) {
-    const int lane = threadIdx.x & 31;
-    uint32_t key[KPL];
-    int pos[KPL];
-#pragma unroll
-    for (int i = 0; i < KPL; i += 4) {
-        const int e = KPL * lane + i;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (e < E) v = __ldcg(reinterpret_cast<const float4 *>(logits + (size_t)t * E + e));  // E % 4 == 0
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            key[i + q] = e + q < E ? ordered_key(vv[q]) : 0u;  // 0: below every real key
-            pos[i + q] = i + q;
-        }
-    }
-#pragma unroll
-    for (int size = 2; size <= KPL; size <<= 1)
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1)
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    // ascending blocks reversed: the network sorts descending by (key, -position)
-                    const bool desc = (i & size) == 0;
-                    const bool jfirst = key[j] > key[i] || (key[j] == key[i] && pos[j] < pos[i]);
-                    const bool sw = desc ? jfirst : !jfirst;
-                    const uint32_t tk = key[i];
-                    const int tp = pos[i];
-                    key[i] = sw ? key[j] : tk;
-                    pos[i] = sw ? pos[j] : tp;
-                    key[j] = sw ? tk : key[j];
-                    pos[j] = sw ? tp : pos[j];
-                }
-            }
-    for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
-        const int wl = __ffs(__ballot_sync(0xffffffffu, key[0] == m)) - 1;
-        const int wp = __shfl_sync(0xffffffffu, pos[0], wl);
-        if (lane == 0) {
-            sel_idx[j] = KPL * wl + wp;
-            sel_val[j] = key_value(m);
-        }
-        if (lane == wl) {
-#pragma unroll
-            for (int i = 0; i + 1 < KPL; ++i) {
-                key[i] = key[i + 1];
-                pos[i] = pos[i + 1];
-            }
-            key[KPL - 1] = 0u;
-        }
-    }
 }
 
 template <int TT>

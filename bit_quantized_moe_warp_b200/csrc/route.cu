@@ -7,6 +7,7 @@
 // over the k selected, and per-expert token lists for the expert kernels.
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace strata {
 
@@ -130,7 +131,17 @@ __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E,
     for (int i = warp; i < kTopkTokensPerCta; i += 8) {
         const int t = t0 + i;
         if (t >= T) break;
-        warp_topk(ws.logits + (size_t)t * E, E, k, s_idx[warp], s_w[warp]);
+        if (E <= 512 && E % 4 == 0) {  // sorted per-lane lists, one warp max + ballot per pick
+            token_topk<16>(ws.logits, t, E, k, s_idx[warp], s_w[warp]);
+            __syncwarp();
+            const float vmax = s_w[warp][0];
+            const float ex = lane < k ? expf(s_w[warp][lane] - vmax) : 0.f;
+            const float den = warp_sum(ex);
+            __syncwarp();
+            if (lane < k) s_w[warp][lane] = ex / den;
+        } else {
+            warp_topk(ws.logits + (size_t)t * E, E, k, s_idx[warp], s_w[warp]);
+        }
         __syncwarp();
         if (lane < k) {
             const int e = s_idx[warp][lane];
