@@ -9,15 +9,18 @@
 // the routing latency once and then keeps the weight stream busy:
 //
 //   phase 0  one warp per CTA starts bulk copies of x and of the CTA's slice
-//            of router rows; the other warps zero the CTA's slice of y,
-//            stage x as fp16 (or bf16(RMSNorm) of the fp32 residual, the
-//            stack glue) and compute the router partial sums of their rows
-//            (fp32, one fixed reduction order per row); grid barrier.
+//            of router rows (the bias comes by cp.async); the other warps
+//            zero the CTA's slice of y, stage x as fp16 (or bf16(RMSNorm) of
+//            the fp32 residual, the stack glue), compute the router partial
+//            sums of their rows in K quarters and reduce them, in a fixed
+//            order, plus the bias, into the logits; grid barrier.
 //   phase 1  every CTA reads all logits and computes, redundantly and
 //            identically, each token's softmax top-k (one warp per token,
-//            warp max reductions, ties to the lower expert index), the
-//            renormalised weights and the per-expert token lists (bit masks
-//            of tokens, popcount ranks). CTA 0 publishes the routing.
+//            per-lane sorted lists, one warp max and a ballot per pick, ties
+//            to the lower expert index), the renormalised weights and the
+//            per-expert token lists (bit masks of tokens, popcount ranks);
+//            warps without a token meanwhile compute the per-block constants
+//            of x. CTA 0 publishes the routing.
 //   phase 2  work units (active expert e, 64-row slice p of its hidden
 //            layer), dealt round-robin over the CTAs. A unit needs no other
 //            unit: it streams the slice's gate and up rows over all of K
@@ -25,10 +28,11 @@
 //            shared memory, then streams the down columns the slice feeds
 //            (contiguous too) and adds w * W_down[:, slice] h into y with
 //            fp32 atomics. One warp per CTA issues 1-D bulk copies of 20 KB
-//            chunks into a ring of shared-memory buffers; 16 warps decode
-//            the 2-bit codes in registers straight into MMA fragments and
-//            multiply on the warp-level MMA (16 rows x 8 tokens x 16
-//            columns, fp16 in, fp32 accumulate).
+//            chunks into a ring of shared-memory buffers and asks L2 for
+//            chunks other CTAs will copy later; 16 warps decode the 2-bit
+//            codes in registers straight into MMA fragments and multiply on
+//            the warp-level MMA (16 rows x 8 tokens x 16 columns, fp16 in,
+//            fp32 accumulate).
 //
 // Exactness of the decode: a code c at mantissa bit p of an fp16 whose
 // exponent gives that bit the place value 1 is the exact value base_p + c
@@ -52,8 +56,8 @@
 namespace strata {
 
 constexpr int kFusedComputeWarps = 16;
-// 16 compute warps + one warp that issues the bulk copies (an issuing thread
-// can stall while the copy engine's queue is full, so no compute warp does).
+// 16 compute warps + one warp that issues the bulk copies, so that copy issue
+// and its waits for free ring buffers never hold up a compute warp.
 constexpr int kFusedThreads = (kFusedComputeWarps + 1) * 32;
 constexpr int kFusedMaxBuf = 16;
 constexpr int kGuSlicesPerChunk = 8;      // gate/up chunk: 8 K-slices x (gate, up) tiles = 20 KB

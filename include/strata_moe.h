@@ -143,9 +143,11 @@ strata_status strata_moe_layer_destroy(strata_moe_layer layer);
  *   router_w    [E x d] fp32, row-major (router bias: desc.router_bias)
  *   expert_blob E packed experts (format above)
  *   y           [n_tokens x d] fp32
- * n_tokens in 0..max_tokens (0 is a no-op). n_tokens <= 16 streams only the
- * selected experts' weights (CUDA cores); larger calls run the grouped
- * tensor-core GEMMs. Errors: INVALID_ARG, TOO_MANY_TOKENS, CUDA. */
+ * n_tokens in 0..max_tokens (0 is a no-op). n_tokens <= 16 runs the whole
+ * layer as one cooperative kernel that streams only the selected experts'
+ * weights (warp-level MMA on codes decoded in registers); larger calls run
+ * the tensor-core router, the routing kernels and the grouped tensor-core
+ * expert GEMMs. Errors: INVALID_ARG, TOO_MANY_TOKENS, CUDA. */
 strata_status strata_moe_forward(strata_moe_layer layer, const void *x_bf16, const float *router_w,
                                  const void *expert_blob, float *y, int32_t n_tokens,
                                  strata_stream_t stream);
@@ -233,8 +235,9 @@ strata_status strata_rmsnorm_bf16(const float *x, void *out_bf16, int32_t n_toke
  * created by the caller. With n_events == 5, every later forward / experts
  * call on this handle records, on its stream: events[0] at its start,
  * [1] after routing, [2] right before and [3] right after the dominant
- * expert kernel (decode: the gate/up streaming kernel; prefill: the gate/up
- * tensor-core GEMM), [4] at its end. n_events == 0 removes the hook.
+ * kernel (decode: the one-launch layer kernel, so [1] coincides with [0];
+ * prefill: the gate/up tensor-core GEMM), [4] at its end. n_events == 0
+ * removes the hook.
  * Errors: INVALID_ARG for any other count. */
 strata_status strata_moe_set_stage_events(strata_moe_layer layer, void *const *events, int32_t n_events);
 
