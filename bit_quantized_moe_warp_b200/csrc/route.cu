@@ -157,7 +157,6 @@ __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E,
 // blk_counts), and the GEMM tile lists: full tiles of all experts first,
 // then the partial ones (largest work first).
 __global__ void __launch_bounds__(1024) k_lists_scan(Workspace ws, int T, int E, int max_tiles1, int max_tiles2) {
-    __shared__ int s_tot[1024];
     __shared__ int s_off[1025];
     __shared__ int s_f1[1025], s_p1[1025], s_f2[1025], s_p2[1025];
     const int nblk = (T + kRouteBlock - 1) / kRouteBlock;
@@ -169,7 +168,6 @@ __global__ void __launch_bounds__(1024) k_lists_scan(Workspace ws, int T, int E,
             ws.blk_counts[(size_t)b * E + e] = tot;  // exclusive prefix over blocks
             tot += c;
         }
-        s_tot[e] = tot;
     }
     // exclusive scans over the experts of: the pair count, the full and the
     // partial gate/up tiles, the full and the partial down tiles (a block
