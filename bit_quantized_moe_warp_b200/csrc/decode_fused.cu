@@ -27,7 +27,7 @@
 //            (contiguous in the blob), forms h = silu(g) * u for the slice in
 //            shared memory, then streams the down columns the slice feeds
 //            (contiguous too) and adds w * W_down[:, slice] h into y with
-//            fp32 atomics. One warp per CTA issues 1-D bulk copies of 20 KB
+//            fp32 atomics. One warp per CTA issues 1-D bulk copies of 40 KB
 //            chunks into a ring of shared-memory buffers and asks L2 for
 //            chunks other CTAs will copy later; 16 warps decode the 2-bit
 //            codes in registers straight into MMA fragments and multiply on
@@ -60,9 +60,13 @@ constexpr int kFusedComputeWarps = 16;
 // and its waits for free ring buffers never hold up a compute warp.
 constexpr int kFusedThreads = (kFusedComputeWarps + 1) * 32;
 constexpr int kFusedMaxBuf = 16;
-constexpr int kGuSlicesPerChunk = 8;      // gate/up chunk: 8 K-slices x (gate, up) tiles = 20 KB
-constexpr int kDownPanelsPerChunk = 16;   // down chunk: 16 tiles of 64 d-rows = 20 KB
-constexpr uint32_t kChunkBytes = 20480;
+// Chunks of 40 KB: every compute warp takes two K slices (or 8 down row
+// groups) per chunk, so the fixed cost of a chunk (all warps waking on its
+// barrier at once, loading the token fragments) is paid half as often as
+// with 20 KB chunks; measured on B200, 4% faster at 1 token, 2.5-4% at 4-16.
+constexpr int kGuSlicesPerChunk = 16;     // gate/up chunk: 16 K-slices x (gate, up) tiles = 40 KB
+constexpr int kDownPanelsPerChunk = 32;   // down chunk: 32 tiles of 64 d-rows = 40 KB
+constexpr uint32_t kChunkBytes = 40960;
 constexpr int kHStride = 64 + 8;          // fp16 row stride of h (halves)
 constexpr int kRouterRowsMax = 16;        // router rows per CTA (E <= 16 * number of CTAs)
 
