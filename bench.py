@@ -36,7 +36,7 @@ METRIC = "MoE layer tokens/s (decode & 8K prefill) + % of HBM / tensor roofline"
 # from one ncu capture (profiles/*.md gives the command). Set to None when the
 # kernel changes after the capture.
 MEASURED_TRAFFIC = {
-    "decode": 19056896,             # k_decode_fused<1>, profiles/decode_fused_T1.md
+    "decode": 19056128,             # k_decode_fused<1>, profiles/decode_fused_T1.md
     "prefill": 683305984,           # k_expert_gemm<0>, profiles/prefill_expert_gemm_8192.md
 }
 PREFILL_KERNELS = 8
