@@ -7,11 +7,13 @@ GEMM, softmax top-k, per-expert lists) and the experts (dequantised 2-bit
 gate/up, SwiGLU, down, weighted combine). Workloads (seeded, synthetic):
   decode        d=2048 f=768 E=512 k=10, 1 token per step, uniform routing (default)
   verify4/16    48-layer stack, 4 or 16 tokens per step, Zipf(1.1) prior
+  verify6       48-layer stack, 1 + 5 drafted tokens per step, Zipf(1.1) prior
+  coder_decode  as decode with 256 experts per layer (the Coder variant)
   prefill       one layer, 8,192-token chunk, Zipf(1.1) prior
   prefill_stack 48 layers, 32,768 tokens in 8,192-token chunks, Zipf(1.1)
-Inputs are resident in HBM before timing; the decode workload rotates over 8
-seeded copies of the layer (6 GB) and 64 token vectors so that no step finds
-its experts in L2. Multi-GPU runs are independent replicas (the layer does
+Inputs are resident in HBM before timing; the single-layer decode workloads
+rotate over 8 seeded copies of the layer (6 GB at 512 experts) and 64 token
+vectors so that no step finds its experts in L2. Multi-GPU runs are independent replicas (the layer does
 not shard); value = units over all ranks / max-over-ranks time.
 """
 from __future__ import annotations
@@ -164,8 +166,10 @@ def run_strata(args, world, rank, local):
     stacked = w.layers > 1
     T = w.T
     chunk = min(T, w.chunk)
-    copies = args.copies if w.name == "decode" else (w.layers if stacked else 1)
-    ntok = 64 if w.name == "decode" else 1
+    rotate = not stacked and T <= 16  # single-layer decode sizes: rotate layer copies and token vectors
+    copies = args.copies if rotate else (w.layers if stacked else 1)
+    ntok = 64 if rotate else 1
+    layer_gb = (w.E * 3 * w.d * w.f // 32 * 10 + w.E * w.d * 4) / 1e9
 
     # inputs (each rank holds its own replica)
     bias_list = [None] * copies
@@ -255,7 +259,7 @@ def run_strata(args, world, rank, local):
     # prefill = router GEMM, top-k, list scan, list scatter, gather, two
     # expert GEMMs; stacks add the RMSNorm kernel per layer and chunk on the
     # prefill path (the decode stack fuses it)
-    launches_per_step = {"decode": 1, "prefill": PREFILL_KERNELS}.get(w.name, None)
+    launches_per_step = 1 if T <= 16 else PREFILL_KERNELS
     if stacked:
         per_layer = 1 if T <= 16 else PREFILL_KERNELS + 1
         launches_per_step = w.layers * per_layer * ((T + chunk - 1) // chunk)
@@ -267,8 +271,8 @@ def run_strata(args, world, rank, local):
         "data": "synthetic (seeded; random-init 2-bit experts)",
         "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
                    "tokens_per_step": T, "layers": w.layers, "routing": "zipf1.1" if w.zipf else "uniform",
-                   "l2": (f"inputs larger than L2: {copies} seeded layer copies ({copies * 0.755:.1f} GB) and 64 token vectors rotated"
-                          if w.name == "decode" else "inputs larger than L2 (0.75 GB per layer)"),
+                   "l2": (f"inputs larger than L2: {copies} seeded layer copies ({copies * layer_gb:.1f} GB) and 64 token vectors rotated"
+                          if rotate else f"inputs larger than L2 ({layer_gb:.2f} GB per layer)"),
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roof,
         "clocks": clk,
@@ -508,15 +512,16 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=["decode", "verify4", "verify16", "prefill",
-                                                              "prefill_stack"])
+                                                              "prefill_stack", "verify6", "coder_decode"])
     ap.add_argument("--impl", default="strata", choices=["strata", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--copies", type=int, default=8, help="decode: seeded layer copies rotated (8 = 6 GB)")
+    ap.add_argument("--copies", type=int, default=8,
+                    help="single-layer decode sizes: seeded layer copies rotated (8 = 6 GB at 512 experts)")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {"decode": 64 * 1024, "verify4": 200, "verify16": 100, "prefill": 200,
-                      "prefill_stack": 3}[args.workload]
+                      "prefill_stack": 3, "verify6": 150, "coder_decode": 64 * 1024}[args.workload]
         if args.impl == "reference":
             args.steps = 3
     world, rank, local = setup_dist(args)

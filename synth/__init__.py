@@ -211,8 +211,12 @@ WORKLOADS = {
     "decode": Workload("decode", 2048, 768, 512, 10, 1, 1, False, 1),
     "verify4": Workload("verify4", 2048, 768, 512, 10, 4, 48, True, 2),
     "verify16": Workload("verify16", 2048, 768, 512, 10, 16, 48, True, 2),
+    # 1 + 5 tokens: a step that verifies the suffix drafter's 5 drafted tokens
+    "verify6": Workload("verify6", 2048, 768, 512, 10, 6, 48, True, 2),
     "prefill": Workload("prefill", 2048, 768, 512, 10, 8192, 1, True, 3),
     "prefill_stack": Workload("prefill_stack", 2048, 768, 512, 10, 32768, 48, True, 4),
+    # the Coder variant of the model keeps 256 of the 512 experts per layer
+    "coder_decode": Workload("coder_decode", 2048, 768, 256, 10, 1, 1, False, 5),
 }
 
 

@@ -232,11 +232,20 @@ def test_decode_layer_full_size():
     print(f"decode T=1: max row err {e:.2e}")
 
 
-@pytest.mark.parametrize("T", [2, 4, 7, 16])
+@pytest.mark.parametrize("T", [2, 4, 6, 7, 16])
 def test_verify_layer_full_size(T):
-    """Decode/verify sizes with the Zipf(1.1) prior, all tokens checked."""
+    """Decode/verify sizes with the Zipf(1.1) prior, all tokens checked
+    (T = 6: one token plus the suffix drafter's five)."""
     e, nex = full_size_check(synth.WORKLOADS["verify4"], T, 0, T)
     print(f"verify T={T}: max row err {e:.2e}, exempt {nex}")
+
+
+@pytest.mark.parametrize("T,sample", [(1, 1), (6, 6), (300, 24)])
+def test_coder_layer_full_size(T, sample):
+    """The Coder variant's layer (256 experts, top-10): decode path at 1 and 6
+    tokens, prefill path at 300."""
+    e, nex = full_size_check(synth.WORKLOADS["coder_decode"], T, 0, sample)
+    print(f"coder T={T}: max row err {e:.2e}, exempt {nex}")
 
 
 @pytest.mark.parametrize("T", [4, 300])
