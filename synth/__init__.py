@@ -211,11 +211,13 @@ WORKLOADS = {
     "decode": Workload("decode", 2048, 768, 512, 10, 1, 1, False, 1),
     "verify4": Workload("verify4", 2048, 768, 512, 10, 4, 48, True, 2),
     "verify16": Workload("verify16", 2048, 768, 512, 10, 16, 48, True, 2),
-    # 1 + 5 tokens: a step that verifies the suffix drafter's 5 drafted tokens
+    # 1 + 5 tokens: a step that verifies the 5 tokens the suffix drafter drafts at once
+    # ("Strata：把 125B 大模型塞进 12GB 显卡…", 再快一截：先猜再验的投机解码)
     "verify6": Workload("verify6", 2048, 768, 512, 10, 6, 48, True, 2),
     "prefill": Workload("prefill", 2048, 768, 512, 10, 8192, 1, True, 3),
     "prefill_stack": Workload("prefill_stack", 2048, 768, 512, 10, 32768, 48, True, 4),
     # the Coder variant of the model keeps 256 of the 512 experts per layer
+    # ("Strata — 8~12GB 显存跑 125B 大模型的本地推理引擎", §5 models table)
     "coder_decode": Workload("coder_decode", 2048, 768, 256, 10, 1, 1, False, 5),
 }
 
