@@ -854,11 +854,13 @@ struct FusedConfig {
     size_t smem;
 };
 
-// Measured on B200: when a block's shared memory forces the largest
-// shared-memory carveout (L1 left with about 28 KB), the MMA loops run about
-// 40% slower than with 150 KB of shared memory. The ring is therefore sized
-// to stay under kFusedSmemSoftCap when that still leaves kFusedMinRing
-// chunks, and only otherwise grows to the device limit.
+// The ring stays under kFusedSmemSoftCap when that still leaves
+// kFusedMinRing chunks, and only otherwise grows to the device limit. The
+// cap comes from a B200 microbenchmark of the MMA loop alone, which ran about
+// 40% slower when the block's shared memory forced the largest carveout (L1
+// left with about 28 KB). In the whole kernel that effect did not show: with
+// 40 KB chunks the default shapes take the device limit (3-5 chunks) and run
+// faster than 20 KB chunks under the cap, and lower caps measured slower.
 constexpr long long kFusedSmemSoftCap = 150 * 1024;
 constexpr int kFusedMinRing = 4;
 
