@@ -43,6 +43,18 @@ MEASURED_TRAFFIC = {
 }
 PREFILL_KERNELS = 8
 
+# default timed steps per workload (each a multiple of the steps one graph replay covers)
+DEFAULT_STEPS = {"decode": 64 * 1024, "verify4": 200, "verify6": 150, "verify16": 100, "prefill": 200,
+                 "prefill_stack": 3, "coder_decode": 64 * 1024}
+
+
+def graph_steps(w) -> int:
+    """Steps one CUDA-graph replay covers: 64 single-layer decode calls, 8
+    prefill chunks, or one whole stack pass (captured by the library)."""
+    if w.layers > 1:
+        return 1
+    return 64 if w.T <= 16 else 8
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -203,7 +215,7 @@ def run_strata(args, world, rank, local):
             handles[c].forward(xs[i % ntok], layers[c].W, layers[c].blob, y, T)
 
     # graph of G steps (a whole stack pass is captured by the library itself)
-    G = (64 if T <= 16 else 8) if not stacked else 1
+    G = graph_steps(w)
     if stacked:
         x_res.copy_(x_stack0)
     for i in range(2):
@@ -291,7 +303,7 @@ def stage_timing(S, w, handles, handle, layers, xs, y, x_res, T, copies, ntok, s
     import torch
     if stacked:
         return None
-    G = 64 if T <= 16 else 8
+    G = graph_steps(w)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(G)]
     for e in evs:
         for ev in e:
@@ -511,8 +523,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=["decode", "verify4", "verify16", "prefill",
-                                                              "prefill_stack", "verify6", "coder_decode"])
+    ap.add_argument("--workload", default="decode", choices=list(DEFAULT_STEPS))
     ap.add_argument("--impl", default="strata", choices=["strata", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -520,8 +531,7 @@ def main():
                     help="single-layer decode sizes: seeded layer copies rotated (8 = 6 GB at 512 experts)")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"decode": 64 * 1024, "verify4": 200, "verify16": 100, "prefill": 200,
-                      "prefill_stack": 3, "verify6": 150, "coder_decode": 64 * 1024}[args.workload]
+        args.steps = DEFAULT_STEPS[args.workload]
         if args.impl == "reference":
             args.steps = 3
     world, rank, local = setup_dist(args)
