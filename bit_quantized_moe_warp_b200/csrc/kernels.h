@@ -107,15 +107,6 @@ inline ExpertStrides expert_strides(const Shape &s) {
                          (size_t)(s.d / 64) * kTileBytes};
 }
 
-// Allow `kernel` the largest dynamic shared memory the device grants a block
-// (max_total, the opt-in limit) minus its static shared memory.
-template <typename Kernel>
-inline cudaError_t set_max_dynamic_smem(Kernel kernel, int max_total) {
-    cudaFuncAttributes a;
-    cudaError_t e = cudaFuncGetAttributes(&a, kernel);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_total - (int)a.sharedSizeBytes);
-}
 size_t down_section_offset(const Shape &s);
 
 }  // namespace strata
