@@ -5,20 +5,26 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl st
 A step is one pass of the hot path over one batch: routing (router GEMV or
 GEMM, softmax top-k, per-expert lists) and the experts (dequantised 2-bit
 gate/up, SwiGLU, down, weighted combine). Workloads (seeded, synthetic):
-  decode        d=2048 f=768 E=512 k=10, 1 token per step, uniform routing (default)
+  decode        d=2048 f=768 E=512 k=10, 1 token per step, uniform routing
+  prefill       one layer, 8,192-token chunk, Zipf(1.1) prior
   verify4/16    48-layer stack, 4 or 16 tokens per step, Zipf(1.1) prior
   verify6       48-layer stack, 1 + 5 drafted tokens per step, Zipf(1.1) prior
   coder_decode  as decode with 256 experts per layer (the Coder variant)
-  prefill       one layer, 8,192-token chunk, Zipf(1.1) prior
   prefill_stack 48 layers, 32,768 tokens in 8,192-token chunks, Zipf(1.1)
+With no --workload the run measures both halves of the metric: the JSON line's
+top level is the one-token decode layer and its "prefill" block the
+8,192-token prefill layer, each timed over exactly --steps steps.
+
 Inputs are resident in HBM before timing; the single-layer decode workloads
 rotate over 8 seeded copies of the layer (6 GB at 512 experts) and 64 token
-vectors so that no step finds its experts in L2. Multi-GPU runs are independent replicas (the layer does
-not shard); value = units over all ranks / max-over-ranks time.
+vectors so that no step finds its experts in L2. Multi-GPU runs are
+independent replicas (the layer does not shard); value = units over all ranks
+/ max-over-ranks time.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -33,27 +39,67 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s (decode & 8K prefill) + % of HBM / tensor roofline"
+CSRC = os.path.join(ROOT, "bit_quantized_moe_warp_b200", "csrc")
 
 # DRAM bytes (read + write) of one launch of each workload's dominant kernel
-# from one ncu capture (profiles/*.md gives the command). Set to None when the
-# kernel changes after the capture.
+# from one ncu capture (the profile under profiles/ gives the command), with
+# the SHA-256 (first 16 hex digits) of the kernel's sources at capture time.
+# When the sources differ the figure no longer describes the kernel and the
+# line reports traffic null.
 MEASURED_TRAFFIC = {
-    "decode": 19056128,             # k_decode_fused<1>, profiles/decode_fused_T1.md
-    "prefill": 683305984,           # k_expert_gemm<0>, profiles/prefill_expert_gemm_8192.md
+    "decode": {"bytes": 19056128, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"),
+               "sha": "unrecorded"},
+    "prefill": {"bytes": 683305984, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "unrecorded"},
 }
-PREFILL_KERNELS = 8
 
-# default timed steps per workload (each a multiple of the steps one graph replay covers)
+# library kernels per single-layer call: decode = the one-launch layer kernel;
+# prefill = W split, router GEMM, top-k, list scan, list scatter, gather, two
+# expert GEMMs, combine
+PREFILL_KERNELS = 9
+DECODE_KERNELS = 1
+
+# default timed steps per workload when --steps is not given
 DEFAULT_STEPS = {"decode": 64 * 1024, "verify4": 200, "verify6": 150, "verify16": 100, "prefill": 200,
                  "prefill_stack": 3, "coder_decode": 64 * 1024}
 
 
 def graph_steps(w) -> int:
-    """Steps one CUDA-graph replay covers: 64 single-layer decode calls, 8
-    prefill chunks, or one whole stack pass (captured by the library)."""
+    """Largest number of steps one CUDA-graph replay covers: 64 single-layer
+    decode calls, 8 prefill chunks, or one whole stack pass (captured by the
+    library itself)."""
     if w.layers > 1:
         return 1
     return 64 if w.T <= 16 else 8
+
+
+def step_plan(steps: int, G: int):
+    """(graph size, replays, remainder): exactly `steps` steps are timed as
+    `replays` replays of a graph of `size` steps plus one replay of a graph of
+    `remainder` steps (0: none)."""
+    if steps < 1:
+        raise ValueError("--steps must be >= 1")
+    size = min(G, steps)
+    reps = steps // size
+    return size, reps, steps - reps * size
+
+
+def sources_sha(names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(CSRC, n), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(name: str):
+    """(bytes, note): the ncu figure of the workload's dominant kernel, or
+    None when there is none or the kernel's sources changed since."""
+    m = MEASURED_TRAFFIC.get(name)
+    if m is None:
+        return None, "no capture"
+    if sources_sha(m["sources"]) != m["sha"]:
+        return None, "kernel changed since the last ncu capture"
+    return m["bytes"], "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"
 
 
 def load_peaks():
@@ -155,155 +201,132 @@ class LayerData:
         self.blob = sd.layer_blob(w, layer_idx, pack)
 
 
-# ---------------------------------------------------------------- workloads
+# ---------------------------------------------------------------- algorithmic units
 
 
-def algorithmic_units(w, route_counts):
-    """Selected-expert bytes of the decode/gate-up stage and expert FLOPs."""
-    d, f = w.d, w.f
-    gu_bytes_per_expert = 2 * d * f // 32 * 10
-    return gu_bytes_per_expert, 2 * 2 * d * f  # bytes per active expert, flops per (token, expert) in gate/up
+def expert_bytes(w) -> int:
+    """Packed bytes of one expert: 3 matrices of d*f weights, 10 bytes per 32."""
+    return 3 * w.d * w.f // 32 * 10
 
 
-def run_strata(args, world, rank, local):
-    import torch
-    import bit_quantized_moe_warp_b200 as S
-    import synth
-    import synth.device as sd
+def decode_bytes(w, n_active):
+    """Algorithmic bytes of one decode-layer launch: the selected experts'
+    packed weights (all three matrices), the router weights and bias, x and y."""
+    return n_active * expert_bytes(w) + w.E * w.d * 4 + w.E * 4 + w.T * w.d * (2 + 4)
 
-    w = synth.WORKLOADS[args.workload]
-    hbm, tf_burst, tf_sust, peak_src = load_peaks()
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-    stacked = w.layers > 1
-    T = w.T
-    chunk = min(T, w.chunk)
-    rotate = not stacked and T <= 16  # single-layer decode sizes: rotate layer copies and token vectors
-    copies = args.copies if rotate else (w.layers if stacked else 1)
-    ntok = 64 if rotate else 1
-    layer_gb = (w.E * 3 * w.d * w.f // 32 * 10 + w.E * w.d * 4) / 1e9
 
-    # inputs (each rank holds its own replica)
-    bias_list = [None] * copies
-    probe = S.MoELayer(w.d, w.f, w.E, w.k, chunk)
-    layers = []
-    for c in range(copies):
-        layers.append(LayerData(S, w, c, probe))
-        bias_list[c] = layers[-1].bias
-    probe.close()
-    if stacked:
-        handle = S.MoELayer(w.d, w.f, w.E, w.k, chunk)
-    else:
-        handle = None
-    xs = sd.x_bf16(w.seed, T * ntok, w.d, stream=rank).view(ntok, T, w.d) if not stacked else None
-    x_stack0 = None
-    if stacked:
-        x_stack0 = sd.x_bf16(w.seed, T, w.d, stream=rank).float()
-    torch.cuda.synchronize()
+def expert_flops(w, tokens) -> int:
+    """Expert FLOPs of `tokens` tokens: k experts x (gate, up, down) x 2 d f."""
+    return tokens * w.k * 6 * w.d * w.f
 
-    # one layer handle per copy for the single-layer workloads (bias lives in the desc)
-    handles = [S.MoELayer(w.d, w.f, w.E, w.k, T, router_bias=layers[c].bias) for c in range(copies)] if not stacked else []
-    y = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
-    x_res = torch.empty((T, w.d), dtype=torch.float32, device=dev) if stacked else None
 
-    def step(i):
-        if stacked:
-            handle.stack_forward([l.W for l in layers], [l.bias for l in layers] if w.zipf else None,
-                                 [l.blob for l in layers], x_res, T, 1e-6)
+# ---------------------------------------------------------------- one workload
+
+
+class Runner:
+    """Inputs, handles and the step function of one workload on this rank."""
+
+    def __init__(self, S, w, rank, copies_arg):
+        import torch
+        import synth.device as sd
+        self.S, self.w = S, w
+        self.dev = torch.device("cuda", torch.cuda.current_device())
+        self.stacked = w.layers > 1
+        self.T = w.T
+        self.chunk = min(w.T, w.chunk)
+        self.rotate = not self.stacked and w.T <= 16
+        self.copies = copies_arg if self.rotate else (w.layers if self.stacked else 1)
+        self.ntok = 64 if self.rotate else 1
+        self.layer_gb = (w.E * expert_bytes(w) + w.E * w.d * 4) / 1e9
+        probe = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk)
+        self.layers = [LayerData(S, w, c, probe) for c in range(self.copies)]
+        probe.close()
+        T = w.T
+        if self.stacked:
+            self.handle = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk)
+            self.handles = []
+            self.x0 = sd.x_bf16(w.seed, T, w.d, stream=rank).float()
+            self.x_res = torch.empty((T, w.d), dtype=torch.float32, device=self.dev)
+            self.xs = None
         else:
-            c = i % copies
-            handles[c].forward(xs[i % ntok], layers[c].W, layers[c].blob, y, T)
+            self.handle = None
+            self.handles = [S.MoELayer(w.d, w.f, w.E, w.k, T, router_bias=self.layers[c].bias)
+                            for c in range(self.copies)]
+            self.xs = sd.x_bf16(w.seed, T * self.ntok, w.d, stream=rank).view(self.ntok, T, w.d)
+            self.x_res = None
+        self.y = torch.zeros((T, w.d), dtype=torch.float32, device=self.dev)
+        torch.cuda.synchronize()
 
-    # graph of G steps (a whole stack pass is captured by the library itself)
-    G = graph_steps(w)
-    if stacked:
-        x_res.copy_(x_stack0)
+    def step(self, i):
+        w = self.w
+        if self.stacked:
+            self.handle.stack_forward([l.W for l in self.layers], [l.bias for l in self.layers] if w.zipf else None,
+                                      [l.blob for l in self.layers], self.x_res, self.T, 1e-6)
+        else:
+            c = i % self.copies
+            self.handles[c].forward(self.xs[i % self.ntok], self.layers[c].W, self.layers[c].blob, self.y, self.T)
+
+    def graph(self, n):
+        """A replay function covering steps 0..n-1 (a CUDA graph for the single
+        layer; the library captures and replays a whole stack pass itself)."""
+        import torch
+        if self.stacked:
+            assert n == 1
+            return lambda: self.step(0)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                self.step(i)
+        self._keep = getattr(self, "_keep", []) + [g]
+        return g.replay
+
+    def close(self):
+        for h in self.handles:
+            h.close()
+        if self.handle is not None:
+            self.handle.close()
+        self.layers = []
+
+
+def time_steps(run, steps, warmup, world):
+    """Exactly `steps` steps timed with CUDA events on the launching stream,
+    after `warmup` untimed ones; returns the max over ranks in ms."""
+    import torch
+    stream = torch.cuda.current_stream()
+    size, reps, rem = step_plan(steps, graph_steps(run.w))
+    if run.stacked:
+        run.x_res.copy_(run.x0)
     for i in range(2):
-        step(i)
+        run.step(i)
     torch.cuda.synchronize()
-    graph = None
-    if not stacked:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for i in range(G):
-                step(i)
-        replay = graph.replay
-    else:
-        replay = lambda: step(0)
-    if args.steps % G:
-        raise SystemExit(f"--steps must be a multiple of {G} for this workload")
-    reps = args.steps // G
-    for _ in range(max(args.warmup, 3)):
-        replay()
+    main = run.graph(size)
+    tail = run.graph(rem) if rem else None
+    for _ in range(-(-max(warmup, 3) // size)):  # at least max(warmup, 3) untimed steps
+        main()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-
-    clocks = Clocks(local)
-    clocks.start()
-    time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(reps):
-        replay()
+        main()
+    if tail is not None:
+        tail()
     e1.record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     barrier(world)
-    ms = dist_max(ms, world)
-    ms_step = ms / args.steps
-    tokens = T * args.steps * world
-    value = tokens / (ms / 1e3)
-    print(f"# timed region: {ms_step * 1e3:.2f} us/step, {value:.1f} tokens/s", file=sys.stderr, flush=True)
-
-    # stage timing of the dominant kernel (separate pass, events around it)
-    dom = stage_timing(S, w, handles, handle, layers, xs, y, x_res, T, copies, ntok, stacked)
-    roof = roofline(w, dom, hbm, tf_burst, peak_src)
-    if stacked and T <= 16:
-        roof = stack_roofline(S, w, layers, x_stack0, T, ms_step, hbm, peak_src)
-
-    # end to end: pinned host input -> device, forward, result -> host, through the API
-    e2e = end_to_end(S, w, handles, handle, layers, T, copies, stacked, world, args)
-
-    # kernels of this library per step: decode = one fused layer kernel;
-    # prefill = router GEMM, top-k, list scan, list scatter, gather, two
-    # expert GEMMs; stacks add the RMSNorm kernel per layer and chunk on the
-    # prefill path (the decode stack fuses it)
-    launches_per_step = 1 if T <= 16 else PREFILL_KERNELS
-    if stacked:
-        per_layer = 1 if T <= 16 else PREFILL_KERNELS + 1
-        launches_per_step = w.layers * per_layer * ((T + chunk - 1) // chunk)
-
-    out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "q2+fp32" if T <= 16 else "q2+fp16->fp32",
-        "data": "synthetic (seeded; random-init 2-bit experts)",
-        "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
-                   "tokens_per_step": T, "layers": w.layers, "routing": "zipf1.1" if w.zipf else "uniform",
-                   "l2": (f"inputs larger than L2: {copies} seeded layer copies ({copies * layer_gb:.1f} GB) and 64 token vectors rotated"
-                          if rotate else f"inputs larger than L2 ({layer_gb:.2f} GB per layer)"),
-                   "parallelism": "replicas" if world > 1 else "single"},
-        "roofline": roof,
-        "clocks": clk,
-        "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps if launches_per_step else None,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+    return dist_max(ms, world), {"graph_steps": size, "replays": reps, "remainder_steps": rem}
 
 
-def stage_timing(S, w, handles, handle, layers, xs, y, x_res, T, copies, ntok, stacked):
-    """Average duration of the dominant expert kernel, from CUDA events the
-    library records around it, over one replay of G steps."""
+def stage_timing(run):
+    """Average duration of the dominant expert kernel (prefill: the gate/up
+    GEMM), from CUDA events the library records around it on the same stream,
+    over one replay of a graph of 8 steps."""
     import torch
-    if stacked:
-        return None
-    G = graph_steps(w)
+    S = run.S
+    G = graph_steps(run.w)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(G)]
     for e in evs:
         for ev in e:
@@ -312,89 +335,166 @@ def stage_timing(S, w, handles, handle, layers, xs, y, x_res, T, copies, ntok, s
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(G):
-            c = i % copies
-            S.strata_moe_set_stage_events(handles[c].handle, evs[i])
-            handles[c].forward(xs[i % ntok], layers[c].W, layers[c].blob, y, T)
-    for h in handles:
+            c = i % run.copies
+            S.strata_moe_set_stage_events(run.handles[c].handle, evs[i])
+            run.step(i)
+    for h in run.handles:
         S.strata_moe_set_stage_events(h.handle, [])
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()
     dom = [evs[i][2].elapsed_time(evs[i][3]) for i in range(G)]
     tot = [evs[i][0].elapsed_time(evs[i][4]) for i in range(G)]
-    # units: selected experts of each step (routing of the last replay)
-    n_active = []
-    for i in range(G):
-        c = i % copies
-        handles[c].forward(xs[i % ntok], layers[c].W, layers[c].blob, y, T)
-        idx = handles[c].routing(T)[0].cpu().numpy()
-        n_active.append(len(set(idx.ravel().tolist())))
-    torch.cuda.synchronize()
-    return {"dom_ms": float(np.mean(dom)), "step_ms": float(np.mean(tot)), "n_active": float(np.mean(n_active)),
-            "T": T}
+    return float(np.mean(dom)), float(np.mean(tot))
 
 
-def decode_bytes(w, n_active):
-    """Algorithmic bytes of one decode-layer launch: the selected experts'
-    packed weights (all three matrices), the router weights and bias, x and y."""
-    return n_active * (3 * w.d * w.f // 32 * 10) + w.E * w.d * 4 + w.E * 4 + w.T * w.d * (2 + 4)
-
-
-def roofline(w, dom, hbm, tf_burst, peak_src):
-    if dom is None:
-        return None
-    if dom["T"] <= 16:
-        bytes_ = decode_bytes(w, dom["n_active"])
-        ach = bytes_ / (dom["dom_ms"] * 1e-3) / 1e9
-        return {"bound": "hbm", "kernel": "k_decode_fused (whole layer, one launch)", "achieved": ach, "peak": hbm,
-                "unit": "GB/s", "frac": ach / hbm, "traffic": MEASURED_TRAFFIC.get(w.name),
-                "algorithmic_bytes_per_launch": bytes_, "selected_experts_per_launch": dom["n_active"],
-                "avg_launch_ms": dom["dom_ms"], "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                "layer_call_ms": dom["step_ms"]}
-    flops = dom["T"] * w.k * 2 * 2 * w.d * w.f
-    ach = flops / (dom["dom_ms"] * 1e-3) / 1e12
-    return {"bound": "tensor", "kernel": "k_expert_gemm<0> (gate/up + SwiGLU)", "achieved": ach, "peak": tf_burst,
-            "unit": "TFLOP/s", "frac": ach / tf_burst, "traffic": MEASURED_TRAFFIC.get(w.name),
-            "algorithmic_flops_per_launch": flops,
-            "avg_launch_ms": dom["dom_ms"], "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops; fp16 same rate)",
-            "layer_call_ms": dom["step_ms"],
-            "layer_expert_TFLOPs": dom["T"] * w.k * 6 * w.d * w.f / (dom["step_ms"] * 1e-3) / 1e12}
-
-
-def stack_roofline(S, w, layers, x0, T, ms_step, hbm, peak_src):
-    """Decode stack: every layer is one fused launch. The selected experts of
-    each layer come from running the same recurrence layer by layer through
-    the library (RMSNorm kernel + fused layer with accumulation) and reading
-    back each layer's routing; achieved = mean algorithmic bytes per layer /
-    (step time / layers)."""
+def active_experts(run, n):
+    """Mean number of distinct selected experts over steps 0..n-1 (routing
+    read back from the library after each call)."""
     import torch
-    dev = torch.cuda.current_device()
-    x = x0.clone()
-    xn = torch.empty((T, w.d), dtype=torch.bfloat16, device=dev)
+    out = []
+    for i in range(n):
+        c = i % run.copies
+        run.step(i)
+        idx = run.handles[c].routing(run.T)[0].cpu().numpy()
+        out.append(len(set(idx.ravel().tolist())))
+    torch.cuda.synchronize()
+    return float(np.mean(out))
+
+
+def stack_active_experts(run):
+    """Distinct selected experts of each layer of a decode stack, from the same
+    recurrence run layer by layer through the library (RMSNorm kernel + layer
+    call with accumulation) and each layer's routing read back."""
+    import torch
+    S, w, T = run.S, run.w, run.T
+    x = run.x0.clone()
+    xn = torch.empty((T, w.d), dtype=torch.bfloat16, device=run.dev)
     n_active = []
     for l in range(w.layers):
         h = S.MoELayer(w.d, w.f, w.E, w.k, T, flags=S.STRATA_ACCUMULATE,
-                       router_bias=layers[l].bias if w.zipf else None)
+                       router_bias=run.layers[l].bias if w.zipf else None)
         S.strata_rmsnorm_bf16(x, xn, T, w.d, 1e-6)
-        h.forward(xn, layers[l].W, layers[l].blob, x, T)
+        h.forward(xn, run.layers[l].W, run.layers[l].blob, x, T)
         idx = h.routing(T)[0].cpu().numpy()
         n_active.append(len(set(idx.ravel().tolist())))
         h.close()
     torch.cuda.synchronize()
-    per_layer_ms = ms_step / w.layers
-    bytes_ = float(np.mean([decode_bytes(w, n) for n in n_active]))
-    ach = bytes_ / (per_layer_ms * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": "k_decode_fused (one launch per layer)", "achieved": ach, "peak": hbm,
-            "unit": "GB/s", "frac": ach / hbm, "traffic": None, "algorithmic_bytes_per_launch": bytes_,
-            "selected_experts_per_launch": float(np.mean(n_active)), "avg_launch_ms": per_layer_ms,
-            "avg_launch_ms_source": "step time / layers (the graph replays one launch per layer)",
+    return n_active
+
+
+def decode_roofline(w, n_active, ms_per_launch, hbm, peak_src, launch_src):
+    """HBM roofline of the one-launch decode layer on the selected experts'
+    packed bytes (router bytes reported beside it)."""
+    sel = n_active * expert_bytes(w)
+    router = w.E * w.d * 4 + w.E * 4
+    alg = decode_bytes(w, n_active)
+    ach = sel / (ms_per_launch * 1e-3) / 1e9
+    traffic, tnote = measured_traffic("decode") if w.name in ("decode",) else (None, "no capture of this shape")
+    return {"bound": "hbm", "kernel": "k_decode_fused (whole layer, one launch)", "achieved": ach, "peak": hbm,
+            "unit": "GB/s", "frac": ach / hbm, "traffic": traffic, "traffic_note": tnote,
+            "bytes_basis": "selected experts' packed weights (gate, up, down)",
+            "selected_expert_bytes_per_launch": sel, "selected_experts_per_launch": n_active,
+            "router_bytes_per_launch": router,
+            "all_algorithmic_bytes_per_launch": alg,
+            "achieved_all_bytes_gbs": alg / (ms_per_launch * 1e-3) / 1e9,
+            "avg_launch_ms": ms_per_launch, "avg_launch_ms_source": launch_src,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"}
 
 
-def end_to_end(S, w, handles, handle, layers, T, copies, stacked, world, args):
+def prefill_roofline(w, dom_ms, layer_ms, peak, peak_src, peak_kind):
+    """Tensor roofline of the gate/up GEMM (the dominant kernel) and of the
+    whole layer on its expert FLOPs."""
+    flops = w.T * w.k * 2 * 2 * w.d * w.f
+    ach = flops / (dom_ms * 1e-3) / 1e12
+    layer = expert_flops(w, w.T) / (layer_ms * 1e-3) / 1e12
+    traffic, tnote = measured_traffic("prefill") if w.name == "prefill" else (None, "no capture of this shape")
+    return {"bound": "tensor", "kernel": "k_expert_gemm<0> (gate/up + SwiGLU)", "achieved": ach, "peak": peak,
+            "unit": "TFLOP/s", "frac": ach / peak, "traffic": traffic, "traffic_note": tnote,
+            "algorithmic_flops_per_launch": flops, "avg_launch_ms": dom_ms,
+            "avg_launch_ms_source": "CUDA events recorded by the library around the kernel, inside the graph",
+            "layer_expert_flops": expert_flops(w, w.T), "layer_ms": layer_ms,
+            "layer_achieved": layer, "layer_frac": layer / peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops {peak_kind}; fp16 kind::f16 runs at the same rate)"}
+
+
+def measure(S, w, args, world, rank, local):
+    """One workload: the timed region, roofline, end-to-end and CPU baseline;
+    returns the JSON block (rank 0's view)."""
     import torch
-    dev = torch.cuda.current_device()
-    if stacked:
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS[w.name]
+    run = Runner(S, w, rank, args.copies)
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms, plan = time_steps(run, steps, args.warmup, world)
+    clk = clocks.stop()
+    ms_step = ms / steps
+    value = w.T * steps * world / (ms / 1e3)
+    print(f"# {w.name}: {ms_step * 1e3:.2f} us/step, {value:.1f} tokens/s", file=sys.stderr, flush=True)
+
+    T = w.T
+    if not run.stacked and T <= 16:
+        n_act = active_experts(run, min(steps, 64))
+        roof = decode_roofline(w, n_act, ms_step, hbm, peak_src,
+                               "graph-timed step (one kernel per step)")
+    elif run.stacked and T <= 16:
+        n_act = stack_active_experts(run)
+        roof = decode_roofline(w, float(np.mean(n_act)), ms_step / w.layers, hbm, peak_src,
+                               "step time / layers (the graph replays one launch per layer)")
+    elif not run.stacked:
+        dom_ms, _ = stage_timing(run)
+        roof = prefill_roofline(w, dom_ms, ms_step, tf_burst, peak_src, "burst")
+    else:
+        layer_ms = ms_step / w.layers / (T // run.chunk)
+        flops = expert_flops(w, run.chunk)
+        ach = flops / (layer_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "whole prefill layer (per 8,192-token chunk)", "achieved": ach,
+                "peak": tf_sust, "unit": "TFLOP/s", "frac": ach / tf_sust, "traffic": None,
+                "traffic_note": "no capture of this shape", "avg_launch_ms": layer_ms,
+                "avg_launch_ms_source": "step time / (layers x chunks)",
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops_sustained)"}
+
+    e2e = end_to_end(run, steps, world)
+    if T <= 16:
+        per_layer = DECODE_KERNELS
+    else:
+        per_layer = PREFILL_KERNELS + (1 if run.stacked else 0)
+    launches = per_layer * w.layers * ((T + run.chunk - 1) // run.chunk) * steps
+    block = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "q2+fp32" if T <= 16 else "q2+fp16->fp32",
+        "data": "synthetic (seeded; random-init 2-bit experts)",
+        "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
+                   "tokens_per_step": T, "layers": w.layers, "routing": "zipf1.1" if w.zipf else "uniform",
+                   "l2": (f"inputs larger than L2: {run.copies} seeded layer copies "
+                          f"({run.copies * run.layer_gb:.1f} GB) and 64 token vectors rotated"
+                          if run.rotate else f"inputs larger than L2 ({run.layer_gb:.2f} GB per layer)"),
+                   "parallelism": "replicas" if world > 1 else "single", "timing": plan},
+        "roofline": roof,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": launches,
+    }
+    run.close()
+    del run
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        block["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    return block
+
+
+def end_to_end(run, steps, world):
+    """The same metric through the public API with host buffers: every step
+    copies that step's x from pinned host memory, runs the layer (or stack)
+    through the C ABI and reads y back into pinned host memory."""
+    import torch
+    S, w, T = run.S, run.w, run.T
+    dev = run.dev
+    if run.stacked:
         xh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
         xh.copy_(torch.randn(T, w.d))
         outh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
@@ -405,18 +505,18 @@ def end_to_end(S, w, handles, handle, layers, T, copies, stacked, world, args):
         outh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
         xd = torch.empty((T, w.d), dtype=torch.bfloat16, device=dev)
     yd = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
-    n = max(8, min(args.steps, 2048 if T <= 16 else 8)) if not stacked else 2
+    n = max(8, min(steps, 2048 if T <= 16 else 8)) if not run.stacked else 2
 
     def one(i):
-        if stacked:
+        if run.stacked:
             xd.copy_(xh, non_blocking=True)
-            handle.stack_forward([l.W for l in layers], [l.bias for l in layers] if w.zipf else None,
-                                 [l.blob for l in layers], xd, T, 1e-6)
+            run.handle.stack_forward([l.W for l in run.layers], [l.bias for l in run.layers] if w.zipf else None,
+                                     [l.blob for l in run.layers], xd, T, 1e-6)
             outh.copy_(xd, non_blocking=True)
         else:
-            c = i % copies
+            c = i % run.copies
             xd.copy_(xh[i % 64], non_blocking=True)
-            handles[c].forward(xd, layers[c].W, layers[c].blob, yd, T)
+            run.handles[c].forward(xd, run.layers[c].W, run.layers[c].blob, yd, T)
             outh.copy_(yd, non_blocking=True)
 
     for i in range(3):
@@ -429,7 +529,7 @@ def end_to_end(S, w, handles, handle, layers, T, copies, stacked, world, args):
     e1.record()
     torch.cuda.synchronize()
     ms = dist_max(e0.elapsed_time(e1), world)
-    h2d = T * w.d * (4 if stacked else 2)
+    h2d = T * w.d * (4 if run.stacked else 2)
     return {"value": T * n * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": T * w.d * 4, "steps": n,
             "note": "pinned host x -> device, forward through the C ABI (Python binding), y -> pinned host"}
@@ -494,46 +594,82 @@ def cpu_baseline(w, seconds):
                       + (f" x{w.layers} layers" if w.layers > 1 else "")}
 
 
-def run_reference(args, world, rank):
-    if rank != 0:
-        return
+def workloads_of(args):
+    """(top-level workload, nested blocks): the default run is the one-token
+    decode layer with the 8,192-token prefill layer nested."""
     import synth
-    w = synth.WORKLOADS[args.workload]
+    if args.workload is None:
+        return synth.WORKLOADS["decode"], [("prefill", synth.WORKLOADS["prefill"])]
+    return synth.WORKLOADS[args.workload], []
+
+
+def reference_block(w, args, world):
+    steps = args.steps if args.steps is not None else 3
     per_step = []
-    budget = args.cpu_seconds / max(1, args.steps + args.warmup)
-    for i in range(args.warmup + args.steps):
+    budget = args.cpu_seconds / max(1, steps + args.warmup)
+    b = None
+    for i in range(args.warmup + steps):
         b = cpu_baseline(w, budget)
         if i >= args.warmup:
             per_step.append(b["value"])
     value = float(np.mean(per_step))
     ms_step = 1e3 * w.T / value
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
-           "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
-                      "tokens_per_step": w.T, "layers": w.layers},
-           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                            "sample": b["sample"]},
-           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
+                       "tokens_per_step": w.T, "layers": w.layers},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {b['sample']}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores on this arm's workloads (rank 0 only)."""
+    if rank != 0:
+        return
+    top, nested = workloads_of(args)
+    out = reference_block(top, args, world)
+    for key, w in nested:
+        # the nested block is one bounded sample (its own cpu_seconds budget)
+        nargs = argparse.Namespace(**vars(args))
+        nargs.steps, nargs.warmup = 1, 0
+        out[key] = reference_block(w, nargs, world)
     print(json.dumps(out), flush=True)
 
 
-def main():
+def run_strata(args, world, rank, local):
+    import bit_quantized_moe_warp_b200 as S
+    top, nested = workloads_of(args)
+    out = measure(S, top, args, world, rank, local)
+    for key, w in nested:
+        out[key] = measure(S, w, args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=list(DEFAULT_STEPS))
+    ap.add_argument("--workload", default=None, choices=list(DEFAULT_STEPS),
+                    help="one workload only (default: decode, with the prefill layer nested)")
     ap.add_argument("--impl", default="strata", choices=["strata", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=8,
                     help="single-layer decode sizes: seeded layer copies rotated (8 = 6 GB at 512 experts)")
-    args = ap.parse_args()
-    if args.steps is None:
-        args.steps = DEFAULT_STEPS[args.workload]
-        if args.impl == "reference":
-            args.steps = 3
+    args = ap.parse_args(argv)
+    if args.steps is not None and args.steps < 1:
+        ap.error("--steps must be >= 1")
+    if args.warmup < 0:
+        ap.error("--warmup must be >= 0")
+    return args
+
+
+def main():
+    args = parse_args()
     world, rank, local = setup_dist(args)
     try:
         if args.impl == "reference":

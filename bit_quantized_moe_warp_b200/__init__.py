@@ -35,7 +35,7 @@ STRATA_FMT_Q2_0_TILED = 1
 STRATA_ACCUMULATE = 1
 STRATA_FORCE_PREFILL = 2
 STRATA_DECODE_MAX_TOKENS = 16
-STRATA_Q2_TILE_BYTES = 2560
+STRATA_Q2_TILE_BYTES = 1280
 
 
 class strata_moe_desc(ctypes.Structure):

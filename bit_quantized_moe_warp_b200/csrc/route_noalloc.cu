@@ -18,14 +18,17 @@
 // each scratch word it later reads, in this call.
 //
 // Set-up: the first call on a device (with that device current) looks up the
-// array's device address with cudaGetSymbolAddress, once, under a lock; the
-// address is kept per device ordinal. That first call can load the module,
-// so it should be made before any stream capture that will contain the call.
+// array's device address with cudaGetSymbolAddress, under a lock; the address
+// is kept per device ordinal together with the context it belongs to, and is
+// looked up again when the current context differs (after a device reset).
+// That first call can load the module, so it should be made before any
+// stream capture that will contain the call.
 //
 // Concurrency: all calls on one device share the one array. Two calls whose
 // work can overlap on the device (different streams without an ordering
 // between them) race on it and give undefined routing; callers serialise
 // them, e.g. by issuing them on one stream.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -65,25 +68,54 @@ __device__ __align__(256) static unsigned char g_route_scratch[kNoallocScratchBy
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
-void *g_scratch_addr[kMaxDevices];
+struct ScratchEntry {
+    CUcontext ctx;  // context the address belongs to
+    void *addr;
+};
+ScratchEntry g_scratch[kMaxDevices];
 
-// Device address of this device's scratch; looked up once per device.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    return fn;
+}
+
+// Device address of this device's scratch in the current context. It is
+// looked up once per (device, context): after a cudaDeviceReset the device's
+// primary context is a new one, the old address is stale, and it is looked
+// up again.
 strata_status scratch_of_current_device(unsigned char **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return strata_set_error(STRATA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices)
         return strata_set_error(STRATA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices - 1);
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return strata_set_error(STRATA_ERR_CUDA, "cuCtxGetCurrent is not available");
+    CUcontext ctx = nullptr;  // null while no context is current on this thread yet
+    if (get(&ctx) != CUDA_SUCCESS) return strata_set_error(STRATA_ERR_CUDA, "cannot read the current CUDA context");
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    ScratchEntry &ent = g_scratch[dev];
+    if (!ent.addr || !ctx || ent.ctx != ctx) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        e = cudaGetSymbolAddress(&p, g_route_scratch);  // makes the primary context current if none is
         if (e != cudaSuccess || !p)
             return strata_set_error(STRATA_ERR_CUDA, "cudaGetSymbolAddress of the routing scratch: %s",
                                     cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx)
+            return strata_set_error(STRATA_ERR_CUDA, "cannot read the current CUDA context");
+        ent.ctx = ctx;
+        ent.addr = p;
     }
-    *out = static_cast<unsigned char *>(g_scratch_addr[dev]);
+    *out = static_cast<unsigned char *>(ent.addr);
     return STRATA_OK;
 }
 
@@ -95,7 +127,12 @@ extern "C" strata_status strata_moe_route_noalloc(const strata_moe_desc *desc, c
                                                   const float *router_w, int32_t n_tokens, int32_t *topk_idx,
                                                   float *topk_w, int32_t *expert_offsets, int32_t *token_list,
                                                   int32_t *pair_slot, strata_stream_t stream) {
-    strata_status s = strata_check_desc(desc);
+    if (!desc) return strata_set_error(STRATA_ERR_INVALID_ARG, "desc is NULL");
+    // max_tokens and flags play no part in this call: check the rest only
+    strata_moe_desc checked = *desc;
+    checked.max_tokens = 1;
+    checked.flags = 0;
+    strata_status s = strata_check_desc(&checked);
     if (s != STRATA_OK) return s;
     if (n_tokens < 0) return strata_set_error(STRATA_ERR_INVALID_ARG, "n_tokens < 0");
     if (n_tokens > kMaxT)

@@ -189,7 +189,8 @@ strata_status strata_moe_get_routing(strata_moe_layer layer, int32_t *topk_idx, 
  * library's own interface.
  *
  * Computes what strata_moe_route computes for desc (router bias from
- * desc->router_bias; max_tokens and flags are ignored) and writes it to the
+ * desc->router_bias; max_tokens and flags are not used and not checked) and
+ * writes it to the
  * caller's device buffers, laid out as strata_moe_get_routing documents:
  * topk_idx [T x k], topk_w [T x k], expert_offsets [E + 1],
  * token_list [T*k], pair_slot [T*k] (all required, 4-byte aligned).
@@ -199,9 +200,10 @@ strata_status strata_moe_get_routing(strata_moe_layer layer, int32_t *topk_idx, 
  * Limit: n_tokens <= STRATA_NOALLOC_MAX_TOKENS (16); larger counts return
  * STRATA_ERR_TOO_MANY_TOKENS. The kernels' scratch is a fixed array of
  * STRATA_NOALLOC_SCRATCH_BYTES in device memory owned by the library, one per
- * device, whose address is looked up by the first call on each device (make
- * that first call before capturing a stream that contains the call). No
- * scratch word needs to start at zero. Calls on one device share that array:
+ * device, whose address is looked up by the first call on each device, and
+ * again after the device's context changes (a cudaDeviceReset); make that
+ * first call before capturing a stream that contains the call. No scratch
+ * word needs to start at zero. Calls on one device share that array:
  * calls whose device work may overlap race on it, so issue them in order
  * (e.g. on one stream). Asynchronous on `stream`. */
 #define STRATA_NOALLOC_MAX_TOKENS 16

@@ -110,3 +110,14 @@ def test_desc_validation(S):
 def test_status_strings(S):
     for code in range(-7, 1):
         assert S.strata_status_string(code)
+
+
+def test_binding_constants_match_header(S):
+    """Every #define the binding restates has the header's value."""
+    src = open(HEADER).read()
+    defs = dict(re.findall(r"#define\s+(STRATA_[A-Z0-9_]+)\s+\(?([0-9]+)u?\b", src))
+    restated = [n for n in dir(S) if n.startswith("STRATA_") and n in defs]
+    assert {"STRATA_Q2_TILE_BYTES", "STRATA_ACCUMULATE", "STRATA_FORCE_PREFILL",
+            "STRATA_DECODE_MAX_TOKENS", "STRATA_FMT_Q2_0_TILED"} <= set(restated)
+    for n in restated:
+        assert getattr(S, n) == int(defs[n]), n

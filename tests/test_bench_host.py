@@ -1,8 +1,10 @@
-"""bench.py's workload table on CPU: every benchmarked workload exists in the
-seeded generators, and every default step count is a whole number of CUDA-graph
-replays (bench.py rejects any other count at run time)."""
+"""bench.py on CPU: the command line the benchmark is run with, the step plan
+that times exactly --steps steps for every workload, and the algorithmic
+units the roofline divides by."""
 import os
 import sys
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -11,11 +13,10 @@ import bench  # noqa: E402
 import synth  # noqa: E402
 
 
-def test_default_steps_cover_whole_graph_replays():
+def test_default_steps_name_generated_workloads():
     for name, steps in bench.DEFAULT_STEPS.items():
         assert name in synth.WORKLOADS, name
-        w = synth.WORKLOADS[name]
-        assert steps > 0 and steps % bench.graph_steps(w) == 0, (name, steps, bench.graph_steps(w))
+        assert steps > 0
 
 
 def test_graph_steps_by_shape():
@@ -27,9 +28,67 @@ def test_graph_steps_by_shape():
         assert bench.graph_steps(W[name]) == 1           # the library captures the whole stack
 
 
+@pytest.mark.parametrize("steps", [1, 3, 7, 8, 9, 20, 63, 64, 65, 100, 200, 64 * 1024, 64 * 1024 + 5])
+def test_step_plan_times_exactly_the_requested_steps(steps):
+    for name, w in synth.WORKLOADS.items():
+        G = bench.graph_steps(w)
+        size, reps, rem = bench.step_plan(steps, G)
+        assert 1 <= size <= G and reps >= 1 and 0 <= rem < size, (name, steps)
+        assert size * reps + rem == steps, (name, steps)
+
+
+def test_driver_command_line_parses_and_plans_every_workload():
+    args = bench.parse_args(["--gpus", "1", "--steps", "20", "--warmup", "5"])
+    assert (args.gpus, args.steps, args.warmup, args.workload, args.impl) == (1, 20, 5, None, "strata")
+    top, nested = bench.workloads_of(args)
+    assert top.name == "decode" and [k for k, _ in nested] == ["prefill"]
+    assert nested[0][1].T == 8192
+    for w in [top] + [v for _, v in nested] + list(synth.WORKLOADS.values()):
+        size, reps, rem = bench.step_plan(args.steps, bench.graph_steps(w))
+        assert size * reps + rem == 20
+    ref = bench.parse_args(["--impl", "reference", "--gpus", "1", "--steps", "20", "--warmup", "5"])
+    assert ref.impl == "reference" and ref.steps == 20
+
+
+def test_bad_step_counts_are_rejected():
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--steps", "0"])
+    with pytest.raises(ValueError):
+        bench.step_plan(0, 64)
+
+
 def test_decode_bytes_counts_selected_experts_router_and_activations():
     w = synth.WORKLOADS["decode"]
     per_expert = 3 * w.d * w.f // 32 * 10                # 2 bits + fp16 scale per 32 weights
-    assert per_expert == 1474560
+    assert per_expert == bench.expert_bytes(w) == 1474560
     assert bench.decode_bytes(w, 10) == 10 * per_expert + w.E * w.d * 4 + w.E * 4 + w.T * w.d * 6
     assert bench.decode_bytes(w, 10) == 18954240
+
+
+def test_decode_roofline_is_on_selected_expert_bytes_over_the_step():
+    w = synth.WORKLOADS["decode"]
+    r = bench.decode_roofline(w, 10.0, 0.01, 6500.0, "fallback", "graph-timed step")
+    assert r["selected_expert_bytes_per_launch"] == 14745600
+    assert abs(r["achieved"] - 14745600 / 1e-5 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6500.0) < 1e-12
+    assert r["router_bytes_per_launch"] == w.E * w.d * 4 + w.E * 4
+
+
+def test_prefill_flops():
+    w = synth.WORKLOADS["prefill"]
+    assert bench.expert_flops(w, w.T) == 8192 * 10 * 6 * 2048 * 768   # 773.1 GFLOP
+    r = bench.prefill_roofline(w, 0.5, 1.0, 1600.0, "fallback", "burst")
+    assert abs(r["layer_achieved"] - 773.094113280) < 1e-6
+    assert abs(r["achieved"] - 515.39607552 / 0.5) < 1e-6
+
+
+def test_traffic_is_dropped_when_kernel_sources_change():
+    m = bench.MEASURED_TRAFFIC["decode"]
+    saved = m["sha"]
+    try:
+        m["sha"] = bench.sources_sha(m["sources"])
+        assert bench.measured_traffic("decode")[0] == m["bytes"]
+        m["sha"] = "0" * 16
+        assert bench.measured_traffic("decode")[0] is None
+    finally:
+        m["sha"] = saved

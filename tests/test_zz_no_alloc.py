@@ -59,6 +59,54 @@ def test_noalloc_routing_matches_layer_routing(T):
         assert np.allclose(got[1].sum(axis=1), 1.0, atol=1e-5)
 
 
+def _compare(got, ref, T, k, what):
+    names = ("topk_idx", "topk_w", "expert_offsets", "token_list", "pair_slot")
+    for name, a, b in zip(names, got, ref):
+        if name == "topk_w":
+            assert np.allclose(a, b, rtol=1e-6, atol=0), f"{what}: {name}"
+        else:
+            assert np.array_equal(a, b), f"{what}: {name}"
+    assert got[2][-1] == T * k, f"{what}: offsets[E] is not T*k"
+    assert np.allclose(got[1].sum(axis=1), 1.0, atol=1e-5)
+
+
+def test_noalloc_routing_at_the_scratch_limits():
+    """The largest shape the fixed scratch is sized for: 16 tokens, 1,024
+    experts, top-32 (the last tile slots and the end of the array; E > 512
+    takes the general warp top-k)."""
+    import torch
+    import synth.device as sd
+    lib = S()
+    w = synth.Workload("limits", 256, 128, 1024, 32, 16, 1, False, 11)
+    W = torch.from_numpy(synth.gen_router_w(w.seed, 0, w.E, w.d)).to(torch_dev())
+    for call in range(2):
+        x = sd.x_bf16(w.seed, w.T, w.d, stream=70 + call)
+        ref = _handle_routing(lib, w, x, W, None, w.T)
+        got = _noalloc_routing(lib, w, x, W, None, w.T)
+        _compare(got, ref, w.T, w.k, f"call {call}")
+
+
+def test_noalloc_routing_ignores_max_tokens_and_flags():
+    import torch
+    import synth.device as sd
+    lib = S()
+    w = synth.WORKLOADS["tiny"]
+    W = torch.from_numpy(synth.gen_router_w(w.seed, 0, w.E, w.d)).to(torch_dev())
+    x = sd.x_bf16(w.seed, w.T, w.d, stream=3)
+    ref = _handle_routing(lib, w, x, W, None, w.T)
+    desc = lib.make_desc(w.d, w.f, w.E, w.k, 0, 0x80)   # max_tokens 0 and an unknown flag: not used here
+    P = w.T * w.k
+    dev = torch_dev()
+    out = [torch.full((w.T, w.k), -7, dtype=torch.int32, device=dev),
+           torch.full((w.T, w.k), -7.0, dtype=torch.float32, device=dev),
+           torch.full((w.E + 1,), -7, dtype=torch.int32, device=dev),
+           torch.full((P,), -7, dtype=torch.int32, device=dev),
+           torch.full((P,), -7, dtype=torch.int32, device=dev)]
+    lib.strata_moe_route_noalloc(desc, x, W, w.T, *out)
+    torch.cuda.synchronize()
+    _compare([a.cpu().numpy() for a in out], ref, w.T, w.k, "max_tokens 0")
+
+
 def test_noalloc_routing_rejects_too_many_tokens():
     import torch
     lib = S()
