@@ -186,4 +186,17 @@ STRATA_DEV float warp_sum(float v) {
 
 STRATA_DEV float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
+// Power-of-two scale of one token's activations for the fp16 operands: s =
+// 2^e with amax * s in [1, 2) (e clamped to [-30, 30], so that 1 / s^2 stays
+// a normal fp32 multiplier; amax == 0 gives 1).
+// Multiplying by s, and later by 1 / s or 1 / s^2, is exact in fp32, so the
+// scaled fp16 operands keep bf16's dynamic range: every element within 2^-14
+// of the token's largest is a normal fp16 number.
+STRATA_DEV float pow2_scale(float amax) {
+    const uint32_t ex = (__float_as_uint(amax) >> 23) & 0xffu;  // amax >= 0
+    int e = amax > 0.f ? 127 - (int)ex : 0;
+    e = e < -30 ? -30 : (e > 30 ? 30 : e);
+    return __uint_as_float((uint32_t)(127 + e) << 23);
+}
+
 }  // namespace strata

@@ -40,8 +40,12 @@
 // accumulates sum_k (base_k + c_k) x_k in fp32; subtracting the per-token
 // constant Z = sum_k base_k x_k + 1.5 sum_k x_k of each 32-column block and
 // multiplying by the block's fp16 scale gives sum_k (c_k - 1.5) s x_k, up to
-// fp32 rounding. x (bf16) is exact in fp16 for |x| in [6.1e-5, 65504]; h is
-// rounded to fp16 (relative error <= 2^-11).
+// fp32 rounding. Each token's x is staged as fp16(x * s) with s = 2^e putting
+// its largest |x| in [1, 2): exact for every element within 2^-14 of that
+// largest, whatever the token's magnitude; the router sums and the gate/up
+// dot products carry s and are divided by it exactly. h, which grows as x^2,
+// is rounded to fp16 as h * s^2 (relative error <= 2^-11) and the down output
+// is divided by s^2.
 //
 // Every wait (grid barrier, copy barrier) is time-bounded; on expiry the
 // kernel records a timeout in the status word and unwinds. Decisions to stop
@@ -69,6 +73,9 @@ constexpr int kDownPanelsPerChunk = 32;   // down chunk: 32 tiles of 64 d-rows =
 constexpr uint32_t kChunkBytes = 40960;
 constexpr int kHStride = 64 + 8;          // fp16 row stride of h (halves)
 constexpr int kRouterRowsMax = 16;        // router rows per CTA (E <= 16 * number of CTAs)
+// room left beside the dynamic shared memory for the kernel's static arrays
+// (barriers, flags, per-token scales, per-pair weights: about 2.7 KB)
+constexpr long long kFusedStaticSmem = 4096;
 
 struct FusedArgs {
     const void *x;        // bf16 [T x d]; fp32 residual [T x d] when rms
@@ -331,6 +338,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar;
     __shared__ int s_abort;
+    // per token: the power-of-two scale s of its staged x and 1 / s (exact);
+    // per sorted pair: the routing weight / s^2 of its token
+    __shared__ float xsc[kDecMaxT], xin[kDecMaxT], pws[kDecMaxT * 32];
     constexpr int NT = TT <= 8 ? 1 : 2;  // MMA n-tiles of 8 token slots
     constexpr int NS = NT * 8;
 
@@ -416,13 +426,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 }
                 ss = warp_sum(ss);
                 const float inv = 1.0f / sqrtf(ss / (float)d + a.eps);
+                float am = 0.f;  // largest |x| of the token, for the scale of the normalised row
+                for (int c = lane; c < d / 4; c += 32) {
+                    const float4 v = xr[c];
+                    am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                }
+                am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(am)));
+                const float sc = pow2_scale(am * inv);
+                if (lane == 0) {
+                    xsc[t] = sc;
+                    xin[t] = 1.0f / sc;
+                }
                 for (int c = lane; c < d / 4; c += 32) {
                     const float4 v = xr[c];
                     __half2 *dst = reinterpret_cast<__half2 *>(xh + (size_t)t * dpx + 4 * c);
-                    dst[0] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.x * inv)),
-                                               __bfloat162float(__float2bfloat16_rn(v.y * inv)));
-                    dst[1] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.z * inv)),
-                                               __bfloat162float(__float2bfloat16_rn(v.w * inv)));
+                    dst[0] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.x * inv)) * sc,
+                                               __bfloat162float(__float2bfloat16_rn(v.y * inv)) * sc);
+                    dst[1] = __floats2half2_rn(__bfloat162float(__float2bfloat16_rn(v.z * inv)) * sc,
+                                               __bfloat162float(__float2bfloat16_rn(v.w * inv)) * sc);
                 }
             }
         } else {
@@ -431,15 +452,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 mbar_wait(&xbar, 0, status, &s_abort);
                 xv = reinterpret_cast<const uint4 *>(bufs);
             }
+            // each token's power-of-two scale (one warp per token: largest |x| from the bf16 bits)
+            for (int t = warp; t < T; t += kFusedComputeWarps) {
+                uint32_t am = 0u;
+                for (int c = lane; c < d / 8; c += 32) {
+                    const uint4 v = xv[(size_t)t * (d / 8) + c];
+                    const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) am = max(am, max(u4[j] & 0x7fffu, (u4[j] >> 16) & 0x7fffu));
+                }
+                am = __reduce_max_sync(0xffffffffu, am);
+                if (lane == 0) {
+                    const float sc = pow2_scale(__uint_as_float(am << 16));
+                    xsc[t] = sc;
+                    xin[t] = 1.0f / sc;
+                }
+            }
+            compute_sync();
             for (int i = tid; i < T * d / 8; i += 512) {
                 const uint4 v = xv[i];
                 const int t = (i * 8) / d, c = (i * 8) % d;
+                const float sc = xsc[t];
                 const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t h4[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const __half2 hv =
-                        __floats2half2_rn(__uint_as_float(u4[j] << 16), __uint_as_float(u4[j] & 0xffff0000u));
+                    const __half2 hv = __floats2half2_rn(__uint_as_float(u4[j] << 16) * sc,
+                                                         __uint_as_float(u4[j] & 0xffff0000u) * sc);
                     h4[j] = *reinterpret_cast<const uint32_t *>(&hv);
                 }
                 *reinterpret_cast<uint4 *>(xh + (size_t)t * dpx + c) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
@@ -496,7 +535,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         for (int i = tid; i < T * nr; i += 512) {  // logits: the K quarters in a fixed order, + bias
             const int t = i / nr, rr = i % nr;
             const float *pq = lsm + ((size_t)t * kRouterRowsMax + rr) * 4;
-            logits[(size_t)t * E + r0 + rr] = (((pq[0] + pq[1]) + pq[2]) + pq[3]) + sbias[rr];
+            // the staged x carries the token's scale s: the sum of the quarters times 1 / s (exact)
+            logits[(size_t)t * E + r0 + rr] = ((((pq[0] + pq[1]) + pq[2]) + pq[3]) * xin[t]) + sbias[rr];
         }
     }
     __syncthreads();
@@ -585,6 +625,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             ptok[pos] = t;
             pslot[pos] = j;
             pw[pos] = sel_w[p];
+            pws[pos] = sel_w[p] * xin[t] * xin[t];  // the down products carry s^2 of the token
             if (b == 0) a.ws.pair_of[p] = pos;
         }
         compute_sync();
@@ -758,7 +799,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                         gs += red[((kg * 2 + 0) * 64 + row) * TT + slot];
                         us += red[((kg * 2 + 1) * 64 + row) * TT + slot];
                     }
-                    h = silu_f(gs) * us;
+                    // gs, us carry the token's scale s; h = silu(g) u is stored as h s^2
+                    // (= silu(gs / s) us s), the down output is divided by s^2
+                    const int tk = ptok[eoff + slot];
+                    h = silu_f(gs * xin[tk]) * us * xsc[tk];
                 }
                 hh[slot * kHStride + row] = __float2half_rn(h);
             }
@@ -787,8 +831,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     }
                     tokA[n] = sa < ecnt ? ptok[eoff + sa] : -1;
                     tokB[n] = sa + 1 < ecnt ? ptok[eoff + sa + 1] : -1;
-                    wA[n] = sa < ecnt ? pw[eoff + sa] : 0.f;
-                    wB[n] = sa + 1 < ecnt ? pw[eoff + sa + 1] : 0.f;
+                    // routing weight / s^2 of the slot's token (h was stored scaled by s^2)
+                    wA[n] = sa < ecnt ? pws[eoff + sa] : 0.f;
+                    wB[n] = sa + 1 < ecnt ? pws[eoff + sa + 1] : 0.f;
                 }
                 for (int i = 0; i < nD; ++i, ++c) {
                     const int bi = c % a.nbuf;
@@ -869,7 +914,7 @@ static FusedConfig fused_config(const Shape &s, int T, int max_smem) {
     const int TT = T <= 1 ? 1 : T <= 4 ? 4 : 16;
     const FusedSmem base = fused_plan(T, TT, s.d, s.E, s.k, 0);
     auto ring = [&](long long limit) {
-        const long long room = limit - 2048 - (long long)base.total;
+        const long long room = limit - kFusedStaticSmem - (long long)base.total;
         const int n = room > 0 ? (int)(room / kChunkBytes) : 0;
         return n > kFusedMaxBuf ? kFusedMaxBuf : n;
     };

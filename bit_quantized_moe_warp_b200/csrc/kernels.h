@@ -25,7 +25,8 @@ struct Workspace {
     int32_t *blk_counts;  // [nblk * E] per 256-token block (prefill lists)
     int32_t *act;         // [E] active experts (decode path)
     float *lpart;         // [16 * E * 4]        fused decode: router logits [T][E]
-    void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill)
+    void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill), token scale applied
+    float *pair_s;        // [T * k]  power-of-two scale of each sorted pair's token (prefill)
     void *hbuf;           // fp16 [T*k * f]       SwiGLU outputs (prefill)
     int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
     int4 *tiles2;         // down GEMM tiles

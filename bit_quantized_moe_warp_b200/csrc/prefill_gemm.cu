@@ -65,6 +65,7 @@ struct GemmArgs {
     const int *n_tiles;
     __half *H;         // MODE 0 output
     __half *O;         // MODE 1 output: W_down h per pair [pairs x d]
+    const float *pair_s;  // MODE 0: power-of-two scale of each pair's token (carried by the gathered x)
     uint32_t *status;
 };
 
@@ -202,10 +203,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     float g[16], u[16];
                     tmem_ld16(trow + c0, g);
                     tmem_ld16(trow + NMAX + c0, u);
+                    // G, U carry the pair's token scale s; H = silu(G / s) U s = h s^2
+                    const float sl = (c0 + (lane & 15) < n) ? a.pair_s[p0 + c0 + (lane & 15)] : 1.f;
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < n) a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i]) * u[i]);
+                    for (int i = 0; i < 16; ++i) {
+                        const float sc = __shfl_sync(0xffffffffu, sl, i);
+                        if (c0 + i < n)
+                            a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i] * (1.0f / sc)) * u[i] * sc);
+                    }
                 } else {
                     float o[16];
                     tmem_ld16(trow + c0, o);
@@ -317,18 +323,22 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
     a.tiles = ws.tiles1;
     a.n_tiles = ws.meta + META_N_TILES1;
     a.H = static_cast<__half *>(ws.hbuf);
+    a.pair_s = ws.pair_s;
     a.status = ws.status;
     (void)max_tiles;
     launch_gemm<0>(maps, a, num_sms, st);
 }
 
-// y[t] (+)= sum_j w_j O[pair_of(t, j)]: one CTA per token, 8 features per thread.
+// y[t] (+)= sum_j w_j O[pair_of(t, j)] / s_t^2: one CTA per token, 8 features
+// per thread (O holds W_down h s_t^2, the token's scale squared).
 __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, const int *__restrict__ pair_of,
-                                                 const float *__restrict__ topk_w, float *__restrict__ y, int d,
-                                                 int k, int accumulate) {
+                                                 const float *__restrict__ topk_w, const float *__restrict__ pair_s,
+                                                 float *__restrict__ y, int d, int k, int accumulate) {
     const int t = blockIdx.x;
     const int *po = pair_of + (size_t)t * k;
     const float *wt = topk_w + (size_t)t * k;
+    const float sc = pair_s[po[0]];  // every pair of the token has its scale
+    const float inv2 = 1.0f / (sc * sc);
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
         float acc[8];
 #pragma unroll
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, c
         for (int j = 0; j < k; ++j) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(O + (size_t)po[j] * d + c));
             const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-            const float w = wt[j];
+            const float w = wt[j] * inv2;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float2 f = __half22float2(h[q]);
@@ -357,7 +367,7 @@ __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, c
 
 void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const Shape &s, cudaStream_t st) {
     if (T <= 0) return;
-    k_combine<<<T, 256, 0, st>>>(static_cast<const __half *>(ws.xp), ws.pair_of, ws.topk_w, y, s.d, s.k,
+    k_combine<<<T, 256, 0, st>>>(static_cast<const __half *>(ws.xp), ws.pair_of, ws.topk_w, ws.pair_s, y, s.d, s.k,
                                  accumulate ? 1 : 0);
 }
 

@@ -275,20 +275,32 @@ __global__ void __launch_bounds__(256) k_lists_scatter(Workspace ws, int T, int 
 }
 
 // ------------------------------------------------------------ gather
-// xp[p] = fp16(x[token_list[p]]): one warp per pair row, 16-byte accesses.
+// xp[p] = fp16(x[t] * s_t) for the pair's token t, with s_t = pow2_scale of
+// the token's largest |x| (recorded in pair_s[p]): one warp per pair row,
+// 16-byte accesses; the second pass re-reads the row from L1.
 __global__ void __launch_bounds__(256) k_gather_xp(const __nv_bfloat16 *__restrict__ x,
                                                     const int *__restrict__ token_list, __half *__restrict__ xp,
-                                                    int npairs, int d) {
+                                                    float *__restrict__ pair_s, int npairs, int d) {
     const int p = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (p >= npairs) return;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)token_list[p] * d);
     uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)p * d);
+    uint32_t am = 0u;  // largest |x| of the row, from the bf16 bits
+    for (int c = lane; c < d / 8; c += 32) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+    }
+    am = __reduce_max_sync(0xffffffffu, am);
+    const float sc = pow2_scale(__uint_as_float(am << 16));
+    if (lane == 0) pair_s[p] = sc;
     for (int c = lane; c < d / 8; c += 32) {
         uint4 v = __ldg(src + c);
         uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            float lo = __uint_as_float(in[q] << 16), hi = __uint_as_float(in[q] & 0xffff0000u);
+            float lo = __uint_as_float(in[q] << 16) * sc, hi = __uint_as_float(in[q] & 0xffff0000u) * sc;
             __half2 h = __floats2half2_rn(lo, hi);
             out[q] = *reinterpret_cast<uint32_t *>(&h);
         }
@@ -321,7 +333,7 @@ void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tile
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st) {
     const int np = T * s.k;
     k_gather_xp<<<(np + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), ws.token_list,
-                                               static_cast<__half *>(ws.xp), np, s.d);
+                                               static_cast<__half *>(ws.xp), ws.pair_s, np, s.d);
 }
 
 }  // namespace strata

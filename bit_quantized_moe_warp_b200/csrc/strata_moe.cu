@@ -102,7 +102,7 @@ static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
-    size_t off[22];
+    size_t off[23];
     size_t total;
     int max_tiles1, max_tiles2;
 };
@@ -115,7 +115,7 @@ static Plan plan_workspace(const strata_moe_desc *d) {
     Plan p{};
     p.max_tiles1 = (int)((P + kGemm1N - 1) / kGemm1N + E);
     p.max_tiles2 = (int)((P + kGemm2N - 1) / kGemm2N + E);
-    const size_t sz[22] = {
+    const size_t sz[23] = {
         256,                                      // 0 status
         64 * 4,                                   // 1 meta
         T * E * 4,                                // 2 logits
@@ -138,9 +138,10 @@ static Plan plan_workspace(const strata_moe_desc *d) {
         (2 + E) * 4,                              // 19 sync
         E * (size_t)s.d * 2,                      // 20 w_hi
         E * (size_t)s.d * 2,                      // 21 w_lo
+        P * 4,                                    // 22 pair_s
     };
     size_t o = 0;
-    for (int i = 0; i < 22; ++i) {
+    for (int i = 0; i < 23; ++i) {
         p.off[i] = o;
         o += (sz[i] + 255) & ~(size_t)255;
     }
@@ -172,6 +173,7 @@ static Workspace carve(uint8_t *base, const Plan &p) {
     w.sync = reinterpret_cast<uint32_t *>(base + p.off[19]);
     w.w_hi = base + p.off[20];
     w.w_lo = base + p.off[21];
+    w.pair_s = reinterpret_cast<float *>(base + p.off[22]);
     return w;
 }
 

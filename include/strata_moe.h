@@ -147,7 +147,10 @@ strata_status strata_moe_layer_destroy(strata_moe_layer layer);
  * layer as one cooperative kernel that streams only the selected experts'
  * weights (warp-level MMA on codes decoded in registers); larger calls run
  * the tensor-core router, the routing kernels and the grouped tensor-core
- * expert GEMMs. Errors: INVALID_ARG, TOO_MANY_TOKENS, CUDA. */
+ * expert GEMMs. Both multiply fp16 operands with fp32 accumulation; each
+ * token's x is scaled by a power of two (its largest |x| to [1, 2)) before
+ * the fp16 conversion and the results are scaled back exactly, so any bf16
+ * magnitude keeps full precision. Errors: INVALID_ARG, TOO_MANY_TOKENS, CUDA. */
 strata_status strata_moe_forward(strata_moe_layer layer, const void *x_bf16, const float *router_w,
                                  const void *expert_blob, float *y, int32_t n_tokens,
                                  strata_stream_t stream);

@@ -137,3 +137,24 @@ def row_errors(y_gpu, y_ref):
     den = np.max(np.abs(y_ref), axis=1)
     den[den == 0] = 1.0
     return np.max(np.abs(y_gpu - y_ref), axis=1) / den
+
+
+WTOL = 1e-5         # renormalised routing weights (fp32 exp / sum against fp64)
+
+
+def weights_check(idx_ref, w_ref, idx_gpu, w_gpu, exempt):
+    """topk_w against the oracle's renormalised softmax weights, matched by
+    expert (the slot order may differ inside near-ties), for every token whose
+    selected set equals the oracle's; the weights sum to 1."""
+    n = 0
+    for t in range(idx_ref.shape[0]):
+        ref = {int(e): float(v) for e, v in zip(idx_ref[t], w_ref[t])}
+        got = {int(e): float(v) for e, v in zip(idx_gpu[t], w_gpu[t])}
+        if set(ref) != set(got):
+            assert exempt[t], f"token {t}: selected experts differ"
+            continue
+        for e, v in ref.items():
+            assert abs(got[e] - v) <= WTOL, f"token {t} expert {e}: weight {got[e]} vs {v}"
+        assert abs(sum(got.values()) - 1.0) <= 1e-5, f"token {t}: weights sum to {sum(got.values())}"
+        n += 1
+    assert n > 0

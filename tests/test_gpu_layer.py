@@ -9,7 +9,7 @@ import pytest
 import oracle
 import synth
 from gpu_harness import (TOL, HostLayer, S, device_blob, expert_source, lists_check, routing_check, row_errors,
-                         torch_dev)
+                         torch_dev, weights_check)
 
 pytestmark = pytest.mark.gpu
 
@@ -189,6 +189,40 @@ def test_zero_tokens_and_too_many():
     layer.close()
 
 
+# ---------------------------------------------------------------- activation range
+
+
+def _scaled_tokens(x_bits, scales):
+    """bf16 tokens with row t multiplied by scales[t] (a power of two, so the
+    bf16 values stay exact); a scale given as (a, b) multiplies the even
+    columns by a and the odd ones by b."""
+    x = synth.bf16_bits_to_f32(x_bits).astype(np.float64)
+    for t, sc in enumerate(scales):
+        if isinstance(sc, tuple):
+            x[t, 0::2] *= sc[0]
+            x[t, 1::2] *= sc[1]
+        else:
+            x[t] *= sc
+    out = synth.f32_to_bf16_bits(x.astype(np.float32))
+    assert np.array_equal(synth.bf16_bits_to_f32(out).astype(np.float64), x), "scaled values must stay exact in bf16"
+    return out
+
+
+@pytest.mark.parametrize("flags", [0, 2], ids=["decode", "prefill"])
+def test_activation_range(flags):
+    """Tokens far outside fp16's normal range: all elements below 6.1e-5
+    (2^-20 and 2^-12 of N(0,1)), large ones (2^12: h ~ x^2 would overflow
+    fp16), and rows whose elements span 2^-20 .. 1. The fp16 operands are
+    exact for these after the per-token power-of-two scaling, so every row
+    meets the usual tolerance on both paths."""
+    base = synth.gen_x_bf16(3, 8, 256)
+    scales = [2.0 ** -20, 2.0 ** -12, 2.0 ** 12, (1.0, 2.0 ** -20), (2.0 ** -16, 2.0 ** -2), 1.0, 2.0 ** 6, 2.0 ** -8]
+    x = _scaled_tokens(base, scales)
+    h = HostLayer(256, 128, 16, 4, 8, seed=3, zipf=True, x=x)
+    err = check_full(h, run_layer(h, flags))
+    print(f"activation range (flags={flags}): max row err {err.max():.2e}")
+
+
 # ---------------------------------------------------------------- full size
 
 
@@ -217,6 +251,7 @@ def full_size_check(w: synth.Workload, T: int, flags: int, sample: int, layer_id
     exempt, bad = routing_check(route["logits"], w.k, idx)
     assert not bad, f"routing differs for tokens {bad[:10]}"
     lists_check(route["idx"], idx, exempt, w.E, off, tl, sl)
+    weights_check(route["idx"], route["w"], idx, wg, exempt)
     rng = np.random.default_rng(T)
     cand = np.nonzero(~exempt)[0]
     toks = np.sort(rng.choice(cand, size=min(sample, cand.size), replace=False))

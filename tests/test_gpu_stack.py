@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_harness import TOL, S, device_blob, expert_source, routing_check, row_errors, torch_dev
+from gpu_harness import TOL, S, device_blob, expert_source, lists_check, routing_check, row_errors, torch_dev
 
 pytestmark = pytest.mark.gpu
 EPS = 1e-6
@@ -85,8 +85,10 @@ def test_small_stack_end_to_end():
     xg = run_stack(layer, Wd, bd, blobs, x0, st.L)
     x = x0.copy()
     clean = np.ones(T, bool)
+    upd_sum = np.zeros(T)  # sum over layers of each row's largest |update|
     for l in range(st.L):
         y, route = oracle_layer_update(x, st.W[l], st.bias[l], st.k, lambda e, l=l: st.experts[l][e])
+        upd_sum += np.max(np.abs(y), axis=1)
         lf = route["logits"].astype(np.float32)
         srt = -np.sort(-lf, axis=1)
         clean &= (srt[:, st.k - 1] - srt[:, st.k]) > 1e-3
@@ -94,17 +96,25 @@ def test_small_stack_end_to_end():
     tot = xg.astype(np.float64) - x0
     ref = x.astype(np.float64) - x0
     err = row_errors(tot[clean], ref[clean])
-    assert clean.sum() >= T // 2 and err.max() <= 5e-3, f"{clean.sum()} clean tokens, max err {err.max():.3e}"
+    # Each layer's update is within TOL of its row maximum (the per-layer gate
+    # above); to first order those errors add up over the layers, so a row of
+    # the summed update x_L - x_0 may be off by TOL * sum_l max|y_l| relative
+    # to max|x_L - x_0|. The bound allows twice that for the propagation of
+    # each layer's error through the later layers' RMSNorm and experts.
+    bound = 2 * TOL * upd_sum[clean] / np.max(np.abs(ref[clean]), axis=1)
+    assert clean.sum() >= T // 2 and np.all(err <= bound), \
+        f"{clean.sum()} clean tokens, max err {err.max():.3e}, bounds {bound.min():.2e}..{bound.max():.2e}"
     layer.close()
 
 
-def test_full_size_verify_stack_teacher_forced():
-    """48 layers, d=2048, f=768, E=512, top-10, Zipf prior, 4 tokens: layers
-    0, 23 and 47 checked against the oracle given the GPU's own input."""
+@pytest.mark.parametrize("T", [4, 16])
+def test_full_size_verify_stack_teacher_forced(T):
+    """48 layers, d=2048, f=768, E=512, top-10, Zipf prior, 4 or 16 tokens:
+    layers 0, 23 and 47 checked against the oracle given the GPU's own input.
+    Each one-layer call goes through the stack's graph capture and replay."""
     import torch
     w = synth.WORKLOADS["verify4"]
     lib = S()
-    T = 4
     layer = lib.MoELayer(w.d, w.f, w.E, w.k, 16)
     import synth.device as sd
     Ws, bs, blobs = [], [], []
@@ -135,7 +145,75 @@ def test_full_size_verify_stack_teacher_forced():
         upd = xl1.astype(np.float64) - xl.astype(np.float64)
         err = row_errors(upd, y_ref)
         assert err[same].max() <= TOL, f"layer {l}: max row error {err[same].max():.3e}"
-        print(f"stack layer {l}: max row err {err.max():.2e}")
+        print(f"stack T={T} layer {l}: max row err {err.max():.2e}")
+    layer.close()
+    del blobs
+    torch.cuda.empty_cache()
+
+
+def test_full_size_prefill_stack_teacher_forced():
+    """The 32,768-token prompt through 48 layers (d=2048, f=768, E=512, top-10,
+    Zipf prior) in 8,192-token chunks, one stack call. For layers 0, 23 and 47
+    the oracle gets the GPU's residual entering the layer (a stack call with
+    that many layers; the prefill path has no atomics, so a shorter run
+    reproduces it exactly) and the library's own RMSNorm of it (the kernel
+    the stack runs), and checks on chunks 0 and 3: the RMSNorm against the
+    oracle's (bf16 bits equal except where the fp32 and fp64 values round
+    differently, then one bf16 step apart), every token's routing under the
+    gap rule, the last chunk's per-expert lists, and the layer's update on
+    sampled tokens."""
+    import torch
+    import synth.device as sd
+    w = synth.WORKLOADS["prefill_stack"]
+    lib = S()
+    T, C = w.T, w.chunk
+    layer = lib.MoELayer(w.d, w.f, w.E, w.k, C)
+    Ws, bs, blobs = [], [], []
+    for l in range(w.layers):
+        Wl, bl = sd.layer_inputs(w, l)
+        Ws.append(Wl)
+        bs.append(bl)
+        blobs.append(device_blob(w, l, layer.desc))
+    x0d = sd.x_bf16(w.seed, T, w.d).float()
+
+    def residual(n_layers):
+        xd = x0d.clone()
+        if n_layers:
+            layer.stack_forward(Ws[:n_layers], bs[:n_layers], blobs[:n_layers], xd, T, EPS)
+            layer.check_status()
+        return xd.cpu().numpy()
+
+    rng = np.random.default_rng(4)
+    for l in (0, 23, 47):
+        xl = residual(l)
+        xl1 = residual(l + 1)
+        # the last call of the second run is chunk 3 at layer l: its routing
+        idx3, w3, off3, tl3, sl3 = (a.cpu().numpy() for a in layer.routing(C))
+        W_h = synth.gen_router_w(w.seed, l, w.E, w.d)
+        b_h = synth.router_bias(w, l)
+        for ch in (0, 3):
+            rows = slice(ch * C, (ch + 1) * C)
+            xin = torch.from_numpy(np.ascontiguousarray(xl[rows])).to(torch_dev())
+            xn_d = torch.empty((C, w.d), dtype=torch.bfloat16, device=torch_dev())
+            lib.strata_rmsnorm_bf16(xin, xn_d, C, w.d, EPS)
+            xn = xn_d.view(torch.int16).cpu().numpy().view(np.uint16)
+            xn_ref = oracle.rmsnorm_bf16(xl[rows].astype(np.float64), EPS)
+            diff = np.abs(xn.astype(np.int32) - xn_ref.astype(np.int32))
+            assert diff.max() <= 1 and (diff > 0).mean() < 1e-3, f"layer {l} chunk {ch}: RMSNorm differs"
+            route = oracle.route_layer(xn, W_h, b_h, w.k)
+            if ch == 3:
+                exempt, bad = routing_check(route["logits"], w.k, idx3)
+                assert not bad, f"layer {l} chunk 3: routing differs for tokens {bad[:10]}"
+                lists_check(route["idx"], idx3, exempt, w.E, off3, tl3, sl3)
+            lf = route["logits"].astype(np.float32)
+            srt = -np.sort(-lf, axis=1)
+            clean = np.nonzero((srt[:, w.k - 1] - srt[:, w.k]) > 1e-4)[0]
+            toks = np.sort(rng.choice(clean, size=8, replace=False))
+            y_ref = oracle.layer_outputs(xn, route, toks, expert_source(w, l))
+            upd = xl1[rows][toks].astype(np.float64) - xl[rows][toks].astype(np.float64)
+            err = row_errors(upd, y_ref)
+            assert err.max() <= TOL, f"layer {l} chunk {ch}: max row error {err.max():.3e}"
+            print(f"prefill stack layer {l} chunk {ch}: max row err {err.max():.2e}")
     layer.close()
     del blobs
     torch.cuda.empty_cache()
