@@ -12,7 +12,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# STRATA_MOE_LIB selects another build of the same library (e.g. an instrumented one)
+# STRATA_MOE_LIB selects another build of the same library (e.g. the checked build,
+# libstrata_moe_checked.so)
 LIB_PATH = os.environ.get("STRATA_MOE_LIB") or os.path.join(_HERE, "libstrata_moe.so")
 
 if not os.path.exists(LIB_PATH):
@@ -30,6 +31,7 @@ STRATA_ERR_OOM = -4
 STRATA_ERR_TOO_MANY_TOKENS = -5
 STRATA_ERR_BAD_BLOB = -6
 STRATA_ERR_TIMEOUT = -7
+STRATA_ERR_BOUNDS = -8
 
 STRATA_FMT_Q2_0_TILED = 1
 STRATA_ACCUMULATE = 1
@@ -73,6 +75,8 @@ _SIGS = {
     "strata_moe_pack_expert": (I32, [DP, V, V, V, V, V, V, V]),
     "strata_moe_pack_expert_device": (I32, [DP, V, V, V, V, V, V, V, V]),
     "strata_selftest_wait_timeout": (I32, [ctypes.c_uint64, V]),
+    "strata_selftest_bounds_check": (I32, [V]),
+    "strata_is_checked_build": (I32, []),
     "strata_status_string": (ctypes.c_char_p, [I32]),
     "strata_last_error": (ctypes.c_char_p, []),
 }
@@ -228,6 +232,14 @@ def strata_moe_pack_expert_device(desc, gc, gs, uc, us, dc, ds, dst, stream=None
 
 def strata_selftest_wait_timeout(timeout_ns, stream=None):
     return _lib.strata_selftest_wait_timeout(int(timeout_ns), _stream(stream))
+
+
+def strata_selftest_bounds_check(stream=None):
+    return _lib.strata_selftest_bounds_check(_stream(stream))
+
+
+def strata_is_checked_build():
+    return _lib.strata_is_checked_build()
 
 
 def strata_status_string(status):

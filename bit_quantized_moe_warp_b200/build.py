@@ -8,6 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libstrata_moe.so")
+# the same sources with every data-derived index bounds-checked into the status word
+OUT_CHECKED = os.path.join(HERE, "libstrata_moe_checked.so")
 SOURCES = ["strata_moe.cu", "route.cu", "decode_fused.cu", "prefill_gemm.cu", "misc.cu", "route_noalloc.cu", "router_gemm.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
@@ -23,15 +25,16 @@ def needs_build(out: str = OUT) -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and not needs_build():
-        return OUT
-    cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", OUT,
-           *[os.path.join(CSRC, s) for s in SOURCES], "-lcudart"]
+def build(verbose: bool = False, force: bool = False, checked: bool = False) -> str:
+    out = OUT_CHECKED if checked else OUT
+    if not force and not needs_build(out):
+        return out
+    cmd = [NVCC, *FLAGS, *(["-DSTRATA_CHECKED"] if checked else []), *(["-Xptxas", "-v"] if verbose else []),
+           "-o", out, *[os.path.join(CSRC, s) for s in SOURCES], "-lcudart"]
     subprocess.run(cmd, check=True)
-    return OUT
+    return out
 
 
 if __name__ == "__main__":
-    build(verbose="-v" in sys.argv, force=True)
-    print(OUT)
+    print(build(verbose="-v" in sys.argv, force=True))
+    print(build(verbose="-v" in sys.argv, force=True, checked=True))

@@ -14,9 +14,10 @@
 namespace strata {
 
 // ---------------------------------------------------------------- status
-// Device status word: 0 = OK; bit 0 = a bounded wait ran out.
+// Device status word: 0 = OK; bit 0 = a bounded wait ran out; bit 1 = a
+// bounds check of the checked build (STRATA_CHECKED) failed.
 // Every spin-wait below gives up after kWaitLimitNs and sets the word.
-enum : uint32_t { kStatusTimeout = 1u };
+enum : uint32_t { kStatusTimeout = 1u, kStatusBounds = 2u };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 STRATA_DEV uint64_t globaltimer() {
@@ -27,6 +28,29 @@ STRATA_DEV uint64_t globaltimer() {
 
 STRATA_DEV void set_status(uint32_t *status, uint32_t bits) {
     if (status) atomicOr(status, bits);
+}
+
+// Bounds checks of the checked build: compiled with -DSTRATA_CHECKED, every
+// index the kernels take from data (an expert, a token, a pair, a list
+// position, a tile) is tested before use; a bad one is recorded in the status
+// word and replaced by `fallback` (or its access skipped), so the kernel
+// neither faults nor traps. In the normal build the checks compile away.
+#ifdef STRATA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+STRATA_DEV bool in_bounds(long long v, long long hi, uint32_t *status) {
+    if (kChecked && (v < 0 || v >= hi)) {
+        set_status(status, kStatusBounds);
+        return false;
+    }
+    return true;
+}
+
+STRATA_DEV int checked_index(int v, int hi, int fallback, uint32_t *status) {
+    return in_bounds(v, hi, status) ? v : fallback;
 }
 
 STRATA_DEV uint32_t smem_u32(const void *p) {
@@ -186,17 +210,21 @@ STRATA_DEV float warp_sum(float v) {
 
 STRATA_DEV float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-// Power-of-two scale of one token's activations for the fp16 operands: s =
-// 2^e with amax * s in [1, 2) (e clamped to [-30, 30], so that 1 / s^2 stays
-// a normal fp32 multiplier; amax == 0 gives 1).
+// Power-of-two scale of one token's activations for the fp16 operands: 1 when
+// the token's largest |x| is in [2^-4, 2^4] (the arithmetic is then the
+// unscaled one), else s = 2^e with amax * s in [1, 2) (e clamped to [-30, 30],
+// so that 1 / s^2 stays a normal fp32 multiplier; amax == 0 gives 1).
 // Multiplying by s, and later by 1 / s or 1 / s^2, is exact in fp32, so the
 // scaled fp16 operands keep bf16's dynamic range: every element within 2^-14
 // of the token's largest is a normal fp16 number.
 STRATA_DEV float pow2_scale(float amax) {
+    if (amax >= 0.0625f && amax <= 16.f) return 1.f;  // already in range: no scaling
     const uint32_t ex = (__float_as_uint(amax) >> 23) & 0xffu;  // amax >= 0
     int e = amax > 0.f ? 127 - (int)ex : 0;
     e = e < -30 ? -30 : (e > 30 ? 30 : e);
     return __uint_as_float((uint32_t)(127 + e) << 23);
 }
+// 1 / s for s = pow2_scale(...) (a power of two): the exponent reflected, exact.
+STRATA_DEV float pow2_inverse(float s) { return __uint_as_float((254u << 23) - __float_as_uint(s)); }
 
 }  // namespace strata

@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 const float sc = pow2_scale(am * inv);
                 if (lane == 0) {
                     xsc[t] = sc;
-                    xin[t] = 1.0f / sc;
+                    xin[t] = pow2_inverse(sc);
                 }
                 for (int c = lane; c < d / 4; c += 32) {
                     const float4 v = xr[c];
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 if (lane == 0) {
                     const float sc = pow2_scale(__uint_as_float(am << 16));
                     xsc[t] = sc;
-                    xin[t] = 1.0f / sc;
+                    xin[t] = pow2_inverse(sc);
                 }
             }
             compute_sync();
@@ -567,7 +567,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             for (int r = warp; r < T; r += kFusedComputeWarps)
                 row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         compute_sync();
-        for (int i = tid; i < T * k; i += 512) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
+        for (int i = tid; i < T * k; i += 512)
+            if (in_bounds(sel_idx[i], E, status)) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
         compute_sync();
         {  // counts and exclusive scans of the counts and of (count > 0), 2 experts per thread
             const int e0 = 2 * tid;
@@ -621,7 +622,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         compute_sync();
         for (int p = tid; p < T * k; p += 512) {  // pairs in (expert, ascending token) order
             const int t = p / k, j = p % k, e = sel_idx[p];
+            if (!in_bounds(e, E, status)) continue;
             const int pos = off[e] + __popc(mask[e] & ((1u << t) - 1u));
+            if (!in_bounds(pos, T * k, status)) continue;
             ptok[pos] = t;
             pslot[pos] = j;
             pw[pos] = sel_w[p];
@@ -657,7 +660,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     const int nq = (n_units > b) ? (n_units - b + G - 1) / G : 0;
     // chunk i of unit u: its source and size
     auto chunk_src = [&](int u, int i, uint32_t &bytes) -> const uint8_t * {
-        const uint8_t *ebase = a.blob + (size_t)act[u / FP] * a.ebytes;
+        const uint8_t *ebase = a.blob + (size_t)checked_index(act[u / FP], E, 0, status) * a.ebytes;
         const int p = u % FP;
         if (i < nG) {
             const int s0 = i * kGuSlicesPerChunk, ns = min(kGuSlicesPerChunk, SLK - s0);
@@ -725,7 +728,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         bool bad = false, stop = false;
         for (int q = 0; q < nq; ++q) {
             const int u = b + q * G;
-            const int e = act[u / FP];
+            const int e = checked_index(act[u / FP], E, 0, status);
             const int ecnt = cnt[e], eoff = off[e];
             const int nta = min((ecnt + 7) / 8, NT);
             // ---- gate / up over all of K
@@ -742,9 +745,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     const int sb = 8 * n + g, sa = 8 * n + 2 * t4;
-                    xb[n] = xh + (size_t)(sb < ecnt ? ptok[eoff + sb] : T) * dpx + 2 * t4;  // T: the zero row
-                    z0[n] = xz + (size_t)(sa < ecnt ? ptok[eoff + sa] : T) * (d / 32);
-                    z1[n] = xz + (size_t)(sa + 1 < ecnt ? ptok[eoff + sa + 1] : T) * (d / 32);
+                    // T: the zero row (empty slots; in the checked build also a bad token)
+                    xb[n] = xh + (size_t)(sb < ecnt ? checked_index(ptok[eoff + sb], T, T, status) : T) * dpx + 2 * t4;
+                    z0[n] = xz + (size_t)(sa < ecnt ? checked_index(ptok[eoff + sa], T, T, status) : T) * (d / 32);
+                    z1[n] = xz + (size_t)(sa + 1 < ecnt ? checked_index(ptok[eoff + sa + 1], T, T, status) : T) * (d / 32);
                 }
                 for (int i = 0; i < nG; ++i, ++c) {
                     const int bi = c % a.nbuf;
@@ -801,7 +805,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     }
                     // gs, us carry the token's scale s; h = silu(g) u is stored as h s^2
                     // (= silu(gs / s) us s), the down output is divided by s^2
-                    const int tk = ptok[eoff + slot];
+                    const int tk = checked_index(ptok[eoff + slot], T, 0, status);
                     h = silu_f(gs * xin[tk]) * us * xsc[tk];
                 }
                 hh[slot * kHStride + row] = __float2half_rn(h);
@@ -829,8 +833,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                         zf[n][blk][0] = hz[sa * 2 + blk];
                         zf[n][blk][1] = hz[(sa + 1) * 2 + blk];
                     }
-                    tokA[n] = sa < ecnt ? ptok[eoff + sa] : -1;
-                    tokB[n] = sa + 1 < ecnt ? ptok[eoff + sa + 1] : -1;
+                    tokA[n] = sa < ecnt ? checked_index(ptok[eoff + sa], T, -1, status) : -1;
+                    tokB[n] = sa + 1 < ecnt ? checked_index(ptok[eoff + sa + 1], T, -1, status) : -1;
                     // routing weight / s^2 of the slot's token (h was stored scaled by s^2)
                     wA[n] = sa < ecnt ? pws[eoff + sa] : 0.f;
                     wB[n] = sa + 1 < ecnt ? pws[eoff + sa + 1] : 0.f;

@@ -27,6 +27,7 @@ struct Workspace {
     float *lpart;         // [16 * E * 4]        fused decode: router logits [T][E]
     void *xp;             // fp16 [T*k * d]       gathered expert inputs (prefill), token scale applied
     float *pair_s;        // [T * k]  power-of-two scale of each sorted pair's token (prefill)
+    float *tok_s;         // [T]      power-of-two scale of each token (prefill)
     void *hbuf;           // fp16 [T*k * f]       SwiGLU outputs (prefill)
     int4 *tiles1;         // gate/up GEMM tiles {expert, pair_start, n, 0}
     int4 *tiles2;         // down GEMM tiles
@@ -64,8 +65,10 @@ void launch_router_gemv(const void *x, const float *W, const float *bias, float 
 void launch_router_tc(const Workspace &ws, const RouterMaps &maps, const float *W, const float *bias, float *logits,
                       int T, const Shape &s, int num_sms, cudaStream_t st);
 cudaError_t init_router_attributes(int max_smem);
+// x_scale_src: the bf16 tokens whose power-of-two scales go to ws.tok_s, or
+// nullptr (routing only)
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
-                        cudaStream_t st);
+                        cudaStream_t st, const void *x_scale_src = nullptr);
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st);
 
 // --- fused decode layer (T <= 16, one cooperative launch)
@@ -77,10 +80,10 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
                                 const Shape &s, int num_sms, int max_smem, cudaStream_t st, cudaEvent_t *ev);
 
 // --- prefill experts (tensor cores)
-void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
+void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles, int T,
                          const Shape &s, int num_sms, cudaStream_t st);
 // writes w * W_down h per pair into ws.xp (fp16 [pairs x d]); launch_combine sums them into y
-void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
+void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles, int T,
                          const Shape &s, int num_sms, cudaStream_t st);
 void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const Shape &s, cudaStream_t st);
 
@@ -89,6 +92,9 @@ void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cud
 void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
                                size_t panel_stride, size_t slice_stride, cudaStream_t st);
 void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st);
+// one index one past the end of a 16-entry array, tested with in_bounds (the
+// access is skipped): the status word records it in the checked build only
+void launch_bounds_selftest(uint32_t *status, cudaStream_t st);
 
 size_t expert_bytes(const Shape &s);
 

@@ -85,3 +85,16 @@ void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st
 }
 
 }  // namespace strata
+
+namespace strata {
+
+__global__ void k_bounds_selftest(uint32_t *status) {
+    __shared__ int arr[16];
+    const int idx = 16 + (int)threadIdx.x;  // one past the end
+    arr[threadIdx.x & 15] = 1;
+    if (in_bounds(idx, 16, status)) arr[idx & 15] += 1;  // never taken in the checked build
+}
+
+void launch_bounds_selftest(uint32_t *status, cudaStream_t st) { k_bounds_selftest<<<1, 1, 0, st>>>(status); }
+
+}  // namespace strata

@@ -66,8 +66,21 @@ struct GemmArgs {
     __half *H;         // MODE 0 output
     __half *O;         // MODE 1 output: W_down h per pair [pairs x d]
     const float *pair_s;  // MODE 0: power-of-two scale of each pair's token (carried by the gathered x)
+    int n_experts, n_pairs;   // bounds of the tile entries (checked build)
     uint32_t *status;
 };
+
+// A tile entry {expert, first pair, pairs, 0}; in the checked build a bad
+// one is recorded and replaced by a harmless tile (expert 0, pairs from 0),
+// the same way in every warp role so the pipelines stay in step.
+template <int NMAX>
+STRATA_DEV int4 tile_at(const GemmArgs &a, int i) {
+    int4 tl = a.tiles[i];
+    const bool ok = in_bounds(tl.x, a.n_experts, a.status) && in_bounds(tl.z - 1, NMAX, a.status) &&
+                    in_bounds(tl.y, a.n_pairs, a.status) && in_bounds((long long)tl.y + tl.z - 1, a.n_pairs, a.status);
+    if (!ok) tl = make_int4(0, 0, a.n_pairs < 16 ? a.n_pairs : 16, 0);
+    return tl;
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_constant__ TmaMaps maps, GemmArgs a) {
@@ -117,7 +130,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
         if (lane == 0) {
             uint32_t it = 0;
             for (int item = blockIdx.x; item < n_items && !*(volatile int *)&s_abort; item += gridDim.x) {
-                const int4 tl = a.tiles[item / a.panels];
+                const int4 tl = tile_at<NMAX>(a, item / a.panels);
                 const int panel = item % a.panels;
                 const int npad = (tl.z + 15) & ~15;
                 const int bsel = npad <= 16 ? 0 : npad <= 32 ? 1 : npad <= 64 ? 2 : npad <= 128 ? 3 : 4;
@@ -153,7 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
             uint32_t it = 0, li = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++li) {
-                const int4 tl = a.tiles[item / a.panels];
+                const int4 tl = tile_at<NMAX>(a, item / a.panels);
                 const int npad = (tl.z + 15) & ~15;
                 const uint32_t idesc = umma_idesc_f16(128, npad);
                 const int acc = li & 1;
@@ -190,7 +203,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
         const int m = 32 * q + lane;
         uint32_t li = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
-            const int4 tl = a.tiles[item / a.panels];
+            const int4 tl = tile_at<NMAX>(a, item / a.panels);
             const int panel = item % a.panels;
             const int acc = li & 1;
             if (!mbar_wait(&accfull[acc], (li >> 1) & 1, a.status, &s_abort)) break;
@@ -205,12 +218,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     tmem_ld16(trow + NMAX + c0, u);
                     // G, U carry the pair's token scale s; H = silu(G / s) U s = h s^2
                     const float sl = (c0 + (lane & 15) < n) ? a.pair_s[p0 + c0 + (lane & 15)] : 1.f;
+                    const bool unit = __all_sync(0xffffffffu, sl == 1.f);  // no token of the chunk scaled
+                    const float il = pow2_inverse(sl);
                     tmem_ld_wait();
+                    if (unit) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float sc = __shfl_sync(0xffffffffu, sl, i);
-                        if (c0 + i < n)
-                            a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i] * (1.0f / sc)) * u[i] * sc);
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < n) a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i]) * u[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float sc = __shfl_sync(0xffffffffu, sl, i), inv = __shfl_sync(0xffffffffu, il, i);
+                            if (c0 + i < n)
+                                a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] =
+                                    __float2half_rn(silu_f(g[i] * inv) * u[i] * sc);
+                        }
                     }
                 } else {
                     float o[16];
@@ -309,7 +331,7 @@ cudaError_t init_gemm_attributes(int max_smem) {
     return cudaFuncSetAttribute(k_expert_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<1>::SMEM);
 }
 
-void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles,
+void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles, int T,
                          const Shape &s, int num_sms, cudaStream_t st) {
     GemmArgs a{};
     a.blob = blob;
@@ -324,6 +346,8 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
     a.n_tiles = ws.meta + META_N_TILES1;
     a.H = static_cast<__half *>(ws.hbuf);
     a.pair_s = ws.pair_s;
+    a.n_experts = s.E;
+    a.n_pairs = T * s.k;
     a.status = ws.status;
     (void)max_tiles;
     launch_gemm<0>(maps, a, num_sms, st);
@@ -333,17 +357,19 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
 // per thread (O holds W_down h s_t^2, the token's scale squared).
 __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, const int *__restrict__ pair_of,
                                                  const float *__restrict__ topk_w, const float *__restrict__ pair_s,
-                                                 float *__restrict__ y, int d, int k, int accumulate) {
+                                                 float *__restrict__ y, int d, int k, int accumulate, int n_pairs,
+                                                 uint32_t *status) {
     const int t = blockIdx.x;
     const int *po = pair_of + (size_t)t * k;
     const float *wt = topk_w + (size_t)t * k;
-    const float sc = pair_s[po[0]];  // every pair of the token has its scale
-    const float inv2 = 1.0f / (sc * sc);
+    const float sc = pair_s[checked_index(po[0], n_pairs, 0, status)];  // every pair of the token has its scale
+    const float inv2 = pow2_inverse(sc * sc);
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
         for (int j = 0; j < k; ++j) {
+            if (!in_bounds(po[j], n_pairs, status)) continue;
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(O + (size_t)po[j] * d + c));
             const __half2 *h = reinterpret_cast<const __half2 *>(&v);
             const float w = wt[j] * inv2;
@@ -368,10 +394,10 @@ __global__ void __launch_bounds__(256) k_combine(const __half *__restrict__ O, c
 void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const Shape &s, cudaStream_t st) {
     if (T <= 0) return;
     k_combine<<<T, 256, 0, st>>>(static_cast<const __half *>(ws.xp), ws.pair_of, ws.topk_w, ws.pair_s, y, s.d, s.k,
-                                 accumulate ? 1 : 0);
+                                 accumulate ? 1 : 0, T * s.k, ws.status);
 }
 
-void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles,
+void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, const TmaMaps &maps, int max_tiles, int T,
                          const Shape &s, int num_sms, cudaStream_t st) {
     GemmArgs a{};
     a.blob = blob;
@@ -386,6 +412,8 @@ void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, con
     a.n_tiles = ws.meta + META_N_TILES2;
     (void)y;
     a.O = static_cast<__half *>(ws.xp);  // the gathered inputs are dead once gate/up has run
+    a.n_experts = s.E;
+    a.n_pairs = T * s.k;
     a.status = ws.status;
     (void)max_tiles;
     launch_gemm<1>(maps, a, num_sms, st);

@@ -122,7 +122,10 @@ __device__ void warp_topk(const float *__restrict__ lrow, int E, int k, int *sel
 // Prefill sizes. (1) top-k per token, one warp per token; expert counts per
 // 256-token block accumulated with atomics (blk_counts zeroed beforehand).
 constexpr int kTopkTokensPerCta = 8;  // one token per warp
-__global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E, int k) {
+// With xs (the bf16 tokens) it also records each token's power-of-two scale
+// for the fp16 expert operands in ws.tok_s.
+__global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, const uint4 *__restrict__ xs, int d, int T, int E,
+                                                     int k) {
     __shared__ int s_idx[8][32];
     __shared__ float s_w[8][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,6 +134,17 @@ __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E,
     for (int i = warp; i < kTopkTokensPerCta; i += 8) {
         const int t = t0 + i;
         if (t >= T) break;
+        if (xs) {  // the token's largest |x| (from the bf16 bits) -> its scale
+            uint32_t am = 0u;
+            for (int c = lane; c < d / 8; c += 32) {
+                const uint4 v = __ldg(xs + (size_t)t * (d / 8) + c);
+                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) am = max(am, max(in[j] & 0x7fffu, (in[j] >> 16) & 0x7fffu));
+            }
+            am = __reduce_max_sync(0xffffffffu, am);
+            if (lane == 0) ws.tok_s[t] = pow2_scale(__uint_as_float(am << 16));
+        }
         if (E <= 512 && E % 4 == 0) {  // sorted per-lane lists, one warp max + ballot per pick
             token_topk<16>(ws.logits, t, E, k, s_idx[warp], s_w[warp]);
             __syncwarp();
@@ -147,7 +161,7 @@ __global__ void __launch_bounds__(256) k_topk_blocks(Workspace ws, int T, int E,
             const int e = s_idx[warp][lane];
             ws.topk_idx[(size_t)t * k + lane] = e;
             ws.topk_w[(size_t)t * k + lane] = s_w[warp][lane];
-            atomicAdd(&ws.blk_counts[(size_t)(t / kRouteBlock) * E + e], 1);
+            if (in_bounds(e, E, ws.status)) atomicAdd(&ws.blk_counts[(size_t)(t / kRouteBlock) * E + e], 1);
         }
         __syncwarp();
     }
@@ -258,15 +272,17 @@ __global__ void __launch_bounds__(256) k_lists_scatter(Workspace ws, int T, int 
     if (t < T)
         for (int j = 0; j < k; ++j) {
             int e = ws.topk_idx[(size_t)t * k + j];
-            atomicOr(&s_bits[e * 8 + (i >> 5)], 1u << (i & 31));
+            if (in_bounds(e, E, ws.status)) atomicOr(&s_bits[e * 8 + (i >> 5)], 1u << (i & 31));
         }
     __syncthreads();
     if (t < T)
         for (int j = 0; j < k; ++j) {
             int e = ws.topk_idx[(size_t)t * k + j];
+            if (!in_bounds(e, E, ws.status)) continue;
             int r = __popc(s_bits[e * 8 + (i >> 5)] & ((1u << (i & 31)) - 1u));
             for (int w = 0; w < (i >> 5); ++w) r += __popc(s_bits[e * 8 + w]);
             int pos = ws.blk_counts[(size_t)blockIdx.x * E + e] + r;
+            if (!in_bounds(pos, (long long)T * k, ws.status)) continue;
             ws.token_list[pos] = t;
             ws.pair_slot[pos] = j;
             ws.pair_w[pos] = ws.topk_w[(size_t)t * k + j];
@@ -275,32 +291,28 @@ __global__ void __launch_bounds__(256) k_lists_scatter(Workspace ws, int T, int 
 }
 
 // ------------------------------------------------------------ gather
-// xp[p] = fp16(x[t] * s_t) for the pair's token t, with s_t = pow2_scale of
-// the token's largest |x| (recorded in pair_s[p]): one warp per pair row,
-// 16-byte accesses; the second pass re-reads the row from L1.
+// xp[p] = fp16(x[t] * s_t) for the pair's token t, with s_t the token's
+// power-of-two scale (tok_s, from the routing), copied to pair_s[p]: one warp
+// per pair row, 16-byte accesses.
 __global__ void __launch_bounds__(256) k_gather_xp(const __nv_bfloat16 *__restrict__ x,
-                                                    const int *__restrict__ token_list, __half *__restrict__ xp,
-                                                    float *__restrict__ pair_s, int npairs, int d) {
+                                                    const int *__restrict__ token_list, const float *__restrict__ tok_s,
+                                                    __half *__restrict__ xp, float *__restrict__ pair_s, int npairs,
+                                                    int d, int T, uint32_t *status) {
     const int p = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (p >= npairs) return;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)token_list[p] * d);
+    const int t = token_list[p];
+    if (!in_bounds(t, T, status)) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d);
     uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)p * d);
-    uint32_t am = 0u;  // largest |x| of the row, from the bf16 bits
+    const float sc = tok_s[t];
+    if (lane == 0) pair_s[p] = sc;
     for (int c = lane; c < d / 8; c += 32) {
         const uint4 v = __ldg(src + c);
         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
-    }
-    am = __reduce_max_sync(0xffffffffu, am);
-    const float sc = pow2_scale(__uint_as_float(am << 16));
-    if (lane == 0) pair_s[p] = sc;
-    for (int c = lane; c < d / 8; c += 32) {
-        uint4 v = __ldg(src + c);
-        uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+        uint32_t out[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            float lo = __uint_as_float(in[q] << 16) * sc, hi = __uint_as_float(in[q] & 0xffff0000u) * sc;
+            const float lo = __uint_as_float(in[q] << 16) * sc, hi = __uint_as_float(in[q] & 0xffff0000u) * sc;
             __half2 h = __floats2half2_rn(lo, hi);
             out[q] = *reinterpret_cast<uint32_t *>(&h);
         }
@@ -322,18 +334,19 @@ void launch_router_gemv(const void *x, const float *W, const float *bias, float 
 }
 
 void launch_route_large(const Workspace &ws, int T, int max_tiles1, int max_tiles2, const Shape &s,
-                        cudaStream_t st) {
+                        cudaStream_t st, const void *x_scale_src) {
     const int nblk = (T + kRouteBlock - 1) / kRouteBlock;
     cudaMemsetAsync(ws.blk_counts, 0, (size_t)nblk * s.E * sizeof(int32_t), st);
-    k_topk_blocks<<<(T + kTopkTokensPerCta - 1) / kTopkTokensPerCta, 256, 0, st>>>(ws, T, s.E, s.k);
+    const uint4 *xs = ws.tok_s ? static_cast<const uint4 *>(x_scale_src) : nullptr;
+    k_topk_blocks<<<(T + kTopkTokensPerCta - 1) / kTopkTokensPerCta, 256, 0, st>>>(ws, xs, s.d, T, s.E, s.k);
     k_lists_scan<<<1, 1024, 0, st>>>(ws, T, s.E, max_tiles1, max_tiles2);
     k_lists_scatter<<<nblk, 256, (size_t)s.E * 8 * sizeof(uint32_t), st>>>(ws, T, s.E, s.k);
 }
 
 void launch_gather_xp(const Workspace &ws, const void *x, int T, const Shape &s, cudaStream_t st) {
     const int np = T * s.k;
-    k_gather_xp<<<(np + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), ws.token_list,
-                                               static_cast<__half *>(ws.xp), ws.pair_s, np, s.d);
+    k_gather_xp<<<(np + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x), ws.token_list, ws.tok_s,
+                                               static_cast<__half *>(ws.xp), ws.pair_s, np, s.d, T, ws.status);
 }
 
 }  // namespace strata

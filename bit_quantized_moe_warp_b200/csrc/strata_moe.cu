@@ -51,6 +51,7 @@ extern "C" const char *strata_status_string(strata_status s) {
         case STRATA_ERR_TOO_MANY_TOKENS: return "too many tokens";
         case STRATA_ERR_BAD_BLOB: return "bad expert blob";
         case STRATA_ERR_TIMEOUT: return "device wait timed out";
+        case STRATA_ERR_BOUNDS: return "bounds check failed";
     }
     return "unknown status";
 }
@@ -102,7 +103,7 @@ static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
-    size_t off[23];
+    size_t off[24];
     size_t total;
     int max_tiles1, max_tiles2;
 };
@@ -115,7 +116,7 @@ static Plan plan_workspace(const strata_moe_desc *d) {
     Plan p{};
     p.max_tiles1 = (int)((P + kGemm1N - 1) / kGemm1N + E);
     p.max_tiles2 = (int)((P + kGemm2N - 1) / kGemm2N + E);
-    const size_t sz[23] = {
+    const size_t sz[24] = {
         256,                                      // 0 status
         64 * 4,                                   // 1 meta
         T * E * 4,                                // 2 logits
@@ -139,9 +140,10 @@ static Plan plan_workspace(const strata_moe_desc *d) {
         E * (size_t)s.d * 2,                      // 20 w_hi
         E * (size_t)s.d * 2,                      // 21 w_lo
         P * 4,                                    // 22 pair_s
+        T * 4,                                    // 23 tok_s
     };
     size_t o = 0;
-    for (int i = 0; i < 23; ++i) {
+    for (int i = 0; i < 24; ++i) {
         p.off[i] = o;
         o += (sz[i] + 255) & ~(size_t)255;
     }
@@ -174,6 +176,7 @@ static Workspace carve(uint8_t *base, const Plan &p) {
     w.w_hi = base + p.off[20];
     w.w_lo = base + p.off[21];
     w.pair_s = reinterpret_cast<float *>(base + p.off[22]);
+    w.tok_s = reinterpret_cast<float *>(base + p.off[23]);
     return w;
 }
 
@@ -427,7 +430,7 @@ static strata_status route_impl(strata_moe_layer L, const void *x, const float *
                                 cudaStream_t st) {
     strata_status s = router_impl(L, x, W, bias, L->ws.logits, T, st);
     if (s != STRATA_OK) return s;
-    launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st);
+    launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st, x);
     return check_launch("routing kernels");
 }
 
@@ -436,9 +439,9 @@ static strata_status experts_impl(strata_moe_layer L, const void *x, const void 
     const uint8_t *b = static_cast<const uint8_t *>(blob);
     launch_gather_xp(L->ws, x, T, L->shape, st);
     stage_mark(L, 2, st);
-    launch_expert_gemm1(L->ws, b, L->maps1, L->plan.max_tiles1, L->shape, L->num_sms, st);
+    launch_expert_gemm1(L->ws, b, L->maps1, L->plan.max_tiles1, T, L->shape, L->num_sms, st);
     stage_mark(L, 3, st);
-    launch_expert_gemm2(L->ws, b, y, L->maps2, L->plan.max_tiles2, L->shape, L->num_sms, st);
+    launch_expert_gemm2(L->ws, b, y, L->maps2, L->plan.max_tiles2, T, L->shape, L->num_sms, st);
     launch_combine(L->ws, y, acc, T, L->shape, st);  // y = (or +=) the sum of each token's k expert outputs
     return check_launch("expert kernels");
 }
@@ -644,6 +647,7 @@ extern "C" strata_status strata_moe_check_status(strata_moe_layer L) {
         cudaMemset(L->ws.sync, 0, (size_t)(2 + L->shape.E) * 4);  // counters of an unwound launch
         return fail(STRATA_ERR_TIMEOUT, "a device wait exceeded its time limit");
     }
+    if (w & kStatusBounds) return fail(STRATA_ERR_BOUNDS, "a bounds check of the checked build failed");
     return STRATA_OK;
 }
 
@@ -660,6 +664,27 @@ extern "C" strata_status strata_selftest_wait_timeout(uint64_t timeout_ns, strat
     if (s == STRATA_OK && cudaMemcpyAsync(&w, status, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
         cudaStreamSynchronize(st) == cudaSuccess) {
         s = (w & kStatusTimeout) ? fail(STRATA_ERR_TIMEOUT, "self-test wait timed out as intended") : STRATA_OK;
+    } else if (s == STRATA_OK) {
+        s = fail(STRATA_ERR_CUDA, "self-test readback failed");
+    }
+    cudaFree(status);
+    return s;
+}
+
+extern "C" int32_t strata_is_checked_build(void) { return kChecked ? 1 : 0; }
+
+extern "C" strata_status strata_selftest_bounds_check(strata_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *status = nullptr;
+    CUDA_TRY(cudaMalloc(&status, 4));
+    cudaMemsetAsync(status, 0, 4, st);
+    launch_bounds_selftest(status, st);
+    strata_status s = check_launch("bounds self-test kernel");
+    uint32_t w = 0;
+    if (s == STRATA_OK && cudaMemcpyAsync(&w, status, 4, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+        cudaStreamSynchronize(st) == cudaSuccess) {
+        s = (w & kStatusBounds) ? fail(STRATA_ERR_BOUNDS, "self-test index out of range, recorded as intended")
+                                : STRATA_OK;
     } else if (s == STRATA_OK) {
         s = fail(STRATA_ERR_CUDA, "self-test readback failed");
     }

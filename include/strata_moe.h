@@ -54,7 +54,8 @@ typedef enum {
     STRATA_ERR_OOM = -4,            /* workspace allocation failed */
     STRATA_ERR_TOO_MANY_TOKENS = -5,/* n_tokens > max_tokens (layer calls) */
     STRATA_ERR_BAD_BLOB = -6,       /* blob pointer or packer input invalid */
-    STRATA_ERR_TIMEOUT = -7         /* a device wait exceeded its time limit */
+    STRATA_ERR_TIMEOUT = -7,        /* a device wait exceeded its time limit */
+    STRATA_ERR_BOUNDS = -8          /* checked build: an index taken from data was out of range */
 } strata_status;
 
 /* ------------------------------------------------------------------ format
@@ -247,7 +248,8 @@ strata_status strata_rmsnorm_bf16(const float *x, void *out_bf16, int32_t n_toke
 strata_status strata_moe_set_stage_events(strata_moe_layer layer, void *const *events, int32_t n_events);
 
 /* Synchronise the layer's stream work and read its device status word
- * (OK, or TIMEOUT if a bounded device wait ran out); clears the word. */
+ * (OK, TIMEOUT if a bounded device wait ran out, BOUNDS if a check of the
+ * checked build failed); clears the word. */
 strata_status strata_moe_check_status(strata_moe_layer layer);
 
 /* Pack one matrix on the HOST: codes [rows x K] one code (0..3) per byte,
@@ -270,6 +272,21 @@ strata_status strata_moe_pack_expert_device(const strata_moe_desc *desc, const u
                                             const uint16_t *up_scales, const uint8_t *down_codes,
                                             const uint16_t *down_scales, void *dst,
                                             strata_stream_t stream);
+
+/* Checked build. The library compiled with -DSTRATA_CHECKED
+ * (libstrata_moe_checked.so) tests every index its kernels take from data
+ * (selected experts, tokens of the per-expert lists, list positions, pair
+ * slots, GEMM tile entries) before using it; a bad index is recorded in the
+ * device status word and the access skipped or redirected to a harmless one,
+ * so a corrupted routing shows up as STRATA_ERR_BOUNDS from
+ * strata_moe_check_status instead of a fault. The normal build compiles the
+ * checks away. Same API and results otherwise.
+ * strata_is_checked_build: 1 for the checked build, 0 otherwise.
+ * strata_selftest_bounds_check: launches a kernel that tests an index one
+ * past the end of an array (and skips that access); synchronous. Returns
+ * STRATA_ERR_BOUNDS in the checked build, STRATA_OK in the normal one. */
+int32_t strata_is_checked_build(void);
+strata_status strata_selftest_bounds_check(strata_stream_t stream);
 
 /* Failure-detection self test: launches a kernel whose bounded wait polls a
  * flag that nothing sets, for timeout_ns nanoseconds (1e3..1e10), then

@@ -121,3 +121,17 @@ def test_binding_constants_match_header(S):
             "STRATA_DECODE_MAX_TOKENS", "STRATA_FMT_Q2_0_TILED"} <= set(restated)
     for n in restated:
         assert getattr(S, n) == int(defs[n]), n
+
+
+def test_checked_build_exports_the_same_calls(S):
+    """The checked build is the same library with bounds checks compiled in:
+    it exports every call the header declares and says which build it is."""
+    import __graft_entry__
+
+    path = __graft_entry__._load_builder().build(checked=True)
+    lib = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(lib, n), f"{n} missing from the checked build"
+    lib.strata_is_checked_build.restype = ctypes.c_int32
+    assert lib.strata_is_checked_build() == 1
+    assert S.strata_is_checked_build() == 0
