@@ -54,16 +54,17 @@ def _bind(lib):
     lib.oracle_fp16_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_double_to_bf16.restype = ctypes.c_uint16
     lib.oracle_double_to_bf16.argtypes = [ctypes.c_double]
-    lib.oracle_dequant.argtypes = [I, I, P, P, P]
+    lib.oracle_dequant.argtypes = [I, I, I, P, P, P]
     lib.oracle_unpack_q2_tiled.argtypes = [I, I, P, ctypes.c_long, ctypes.c_long, P, P]
+    lib.oracle_unpack_q4_tiled.argtypes = [I, I, P, ctypes.c_long, ctypes.c_long, P, P]
     lib.oracle_router_logits.argtypes = [I, I, I, P, P, P, P]
     lib.oracle_topk_softmax.argtypes = [I, I, I, P, P, P]
     lib.oracle_expert_lists.argtypes = [I, I, I, P, P, P, P]
-    lib.oracle_expert_ffn.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
-    lib.oracle_moe_layer.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
+    lib.oracle_expert_ffn.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P]
+    lib.oracle_moe_layer.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.oracle_rmsnorm_bf16.argtypes = [I, P, ctypes.c_double, P]
     lib.oracle_residual_add_f32.argtypes = [I, P, P]
-    for fn in ("oracle_dequant", "oracle_unpack_q2_tiled", "oracle_router_logits",
+    for fn in ("oracle_dequant", "oracle_unpack_q2_tiled", "oracle_unpack_q4_tiled", "oracle_router_logits",
                "oracle_topk_softmax", "oracle_expert_lists", "oracle_expert_ffn",
                "oracle_moe_layer", "oracle_rmsnorm_bf16", "oracle_residual_add_f32"):
         getattr(lib, fn).restype = None
@@ -97,12 +98,13 @@ def double_to_bf16(v):
     return np.array([lib.oracle_double_to_bf16(float(x)) for x in np.ravel(v)], dtype=np.uint16).reshape(np.shape(v))
 
 
-def dequant(codes, scales_fp16):
+def dequant(codes, scales_fp16, bits: int = 2):
+    """(c - (2^bits - 1)/2) * scale of the 32-column block, in double."""
     codes = _c(codes, np.uint8)
     sc = _c(np.asarray(scales_fp16).view(np.uint16) if np.asarray(scales_fp16).dtype == np.float16 else scales_fp16, np.uint16)
     rows, K = codes.shape
     W = np.empty((rows, K), dtype=np.float64)
-    load().oracle_dequant(rows, K, _p(codes), _p(sc), _p(W))
+    load().oracle_dequant(rows, K, bits, _p(codes), _p(sc), _p(W))
     return W
 
 
@@ -120,16 +122,32 @@ def unpack_q2_tiled(blob, rows: int, K: int, panel_stride: int = None, slice_str
     return codes, scales.view(np.float16)
 
 
-def unpack_expert(blob, d: int, f: int) -> dict:
+def unpack_q4_tiled(blob, rows: int, K: int, panel_stride: int = None, slice_stride: int = 2304):
+    """Codes and scales of one 4-bit matrix (2304-byte tiles) whose tile
+    (p, s) starts at ``blob + p * panel_stride + s * slice_stride``."""
+    blob = _c(blob, np.uint8)
+    if panel_stride is None:
+        panel_stride = (K // 64) * slice_stride
+    last = (rows // 64 - 1) * panel_stride + (K // 64 - 1) * slice_stride
+    assert blob.size >= last + 2304, "blob too small for rows x K"
+    codes = np.empty((rows, K), dtype=np.uint8)
+    scales = np.empty((rows, K // 32), dtype=np.uint16)
+    load().oracle_unpack_q4_tiled(rows, K, _p(blob), panel_stride, slice_stride, _p(codes), _p(scales))
+    return codes, scales.view(np.float16)
+
+
+def unpack_expert(blob, d: int, f: int, bits: int = 2) -> dict:
     """Codes/scales of one expert from its blob section (header's layout):
     gate/up tiles interleaved in (f-panel, d-slice) order, 2560-byte pairs;
     then the down matrix [d x f] with its tiles in (f-slice, d-panel) order."""
     blob = _c(blob, np.uint8)
-    gu = f * d // 64 * 20 * 2
-    gc, gs = unpack_q2_tiled(blob, f, d, (d // 64) * 2560, 2560)
-    uc, us = unpack_q2_tiled(blob[1280:], f, d, (d // 64) * 2560, 2560)
-    dc, ds = unpack_q2_tiled(blob[gu:], d, f, 1280, (d // 64) * 1280)
-    return dict(gate_codes=gc, gate_scales=gs, up_codes=uc, up_scales=us, down_codes=dc, down_scales=ds)
+    tb = 1280 if bits == 2 else 2304  # tile bytes
+    un = unpack_q2_tiled if bits == 2 else unpack_q4_tiled
+    gu = (f // 64) * (d // 64) * 2 * tb
+    gc, gs = un(blob, f, d, (d // 64) * 2 * tb, 2 * tb)
+    uc, us = un(blob[tb:], f, d, (d // 64) * 2 * tb, 2 * tb)
+    dc, ds = un(blob[gu:], d, f, tb, (d // 64) * tb)
+    return dict(gate_codes=gc, gate_scales=gs, up_codes=uc, up_scales=us, down_codes=dc, down_scales=ds, bits=bits)
 
 
 def router_logits(x_bf16, W, bias=None):
@@ -168,7 +186,8 @@ def _sc(a):
 
 
 def expert_ffn(X, ex: dict):
-    """SwiGLU expert on rows of X (double [n, d]); ex holds codes/scales."""
+    """SwiGLU expert on rows of X (double [n, d]); ex holds codes/scales (and
+    "bits", 2 when absent)."""
     X = _c(X, np.float64)
     n, d = X.shape
     f = ex["gate_codes"].shape[0]
@@ -176,7 +195,7 @@ def expert_ffn(X, ex: dict):
     keep = [_c(ex["gate_codes"], np.uint8), _sc(ex["gate_scales"]),
             _c(ex["up_codes"], np.uint8), _sc(ex["up_scales"]),
             _c(ex["down_codes"], np.uint8), _sc(ex["down_scales"])]
-    load().oracle_expert_ffn(d, f, n, _p(X), *[_p(a) for a in keep], _p(out))
+    load().oracle_expert_ffn(d, f, n, int(ex.get("bits", 2)), _p(X), *[_p(a) for a in keep], _p(out))
     return out
 
 
@@ -205,7 +224,9 @@ def moe_layer(x_bf16, W, bias, experts: list, k: int):
     y = np.empty((T, d), dtype=np.float64)
     idx = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
-    load().oracle_moe_layer(T, d, f, E, k, _p(x), _p(W), _p(b),
+    bits = int(experts[0].get("bits", 2))
+    assert all(int(e.get("bits", 2)) == bits for e in experts), "one code width per layer"
+    load().oracle_moe_layer(T, d, f, E, k, bits, _p(x), _p(W), _p(b),
                             *[ctypes.cast(p, ctypes.c_void_p) for p in pa], _p(y), _p(idx), _p(w))
     return y, idx, w
 

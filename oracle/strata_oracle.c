@@ -29,6 +29,12 @@
  *    the reduction dimension, code c in {0,1,2,3} meaning (c - 1.5) * scale,
  *    one fp16 scale per block. The pages name this format "Q2_0"
  *    ("Strata Skill…", 功能与原则) but do not give its bits.
+ *  - The wider levels of the pages' quality ladder (Q2_0, IQ2_XS, IQ3_XXS,
+ *    IQ3_S: "Strata：把 125B 大模型塞进 12GB 显卡…", 能跑多快 table) trade memory
+ *    for accuracy. Their lattice codebooks are not on the pages; the 4-bit
+ *    block format here is the same rule with 4-bit codes: c in {0..15}
+ *    meaning (c - 7.5) * scale, one fp16 scale per 32 weights. In general a
+ *    b-bit code means c - (2^b - 1) / 2, centred on zero.
  *
  * Readings taken where the pages are silent (each also listed in the design
  * notes): the top-k order key is the logit rounded to fp32 (the precision the
@@ -86,16 +92,18 @@ uint16_t oracle_double_to_bf16(double v)
 
 /* ------------------------------------------------------ format (dequant) */
 
-/* W[r][k] = (c[r][k] - 1.5) * scale[r][k/32]; codes one per byte, row-major
- * [rows x K]; scales fp16 bits, row-major [rows x K/32]. */
-void oracle_dequant(int rows, int K, const uint8_t *codes, const uint16_t *scales, double *W)
+/* W[r][k] = (c[r][k] - (2^bits - 1) / 2) * scale[r][k/32] (bits 2: c - 1.5,
+ * bits 4: c - 7.5); codes one per byte, row-major [rows x K]; scales fp16
+ * bits, row-major [rows x K/32]. */
+void oracle_dequant(int rows, int K, int bits, const uint8_t *codes, const uint16_t *scales, double *W)
 {
     int nb = K / 32;
+    double offset = ((double)(1 << bits) - 1.0) / 2.0;
     for (int r = 0; r < rows; ++r)
         for (int k = 0; k < K; ++k) {
             double s = oracle_fp16_to_double(scales[(size_t)r * nb + k / 32]);
             double c = (double)codes[(size_t)r * K + k];
-            W[(size_t)r * K + k] = (c - 1.5) * s;
+            W[(size_t)r * K + k] = (c - offset) * s;
         }
 }
 
@@ -127,6 +135,38 @@ void oracle_unpack_q2_tiled(int rows, int K, const uint8_t *blob, long panel_str
                 }
                 for (int b = 0; b < 2; ++b) {
                     const uint8_t *sp = tile + 1024 + 4 * i + 2 * b;
+                    scales[(size_t)r * (K / 32) + 2 * s + b] = (uint16_t)(sp[0] | (sp[1] << 8));
+                }
+            }
+        }
+}
+
+/* The 4-bit tiled layout the library's header documents: 64-row x 64-column
+ * tiles of 2304 bytes; inside a tile, row i's 64 codes occupy bytes
+ * 32i..32i+31 as eight little-endian 32-bit words W0..W7, column
+ * c = 16j + 8s + 2t + e of the tile (j < 4, s < 2, t < 4, e < 2) sitting in
+ * word W(2t + j/2) at bit 16e + 8(j % 2) + 4s (four bits); the row's two
+ * fp16 scales (columns 0-31, then 32-63) follow at byte 2048 + 4i. Tiles are
+ * placed as for the 2-bit layout (a lone matrix: slice_stride 2304,
+ * panel_stride (K/64) * 2304). */
+void oracle_unpack_q4_tiled(int rows, int K, const uint8_t *blob, long panel_stride, long slice_stride,
+                            uint8_t *codes, uint16_t *scales)
+{
+    for (int p = 0; p < rows / 64; ++p)
+        for (int s = 0; s < K / 64; ++s) {
+            const uint8_t *tile = blob + (size_t)p * (size_t)panel_stride + (size_t)s * (size_t)slice_stride;
+            for (int i = 0; i < 64; ++i) {
+                int r = p * 64 + i;
+                for (int c = 0; c < 64; ++c) {
+                    int j = c / 16, sh = (c / 8) % 2, t = (c % 8) / 2, e = c % 2;
+                    const uint8_t *wp = tile + 32 * i + 4 * (2 * t + j / 2);
+                    uint32_t w = (uint32_t)wp[0] | ((uint32_t)wp[1] << 8) |
+                                 ((uint32_t)wp[2] << 16) | ((uint32_t)wp[3] << 24);
+                    int bit = 16 * e + 8 * (j % 2) + 4 * sh;
+                    codes[(size_t)r * K + 64 * s + c] = (uint8_t)((w >> bit) & 15u);
+                }
+                for (int b = 0; b < 2; ++b) {
+                    const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;
                     scales[(size_t)r * (K / 32) + 2 * s + b] = (uint16_t)(sp[0] | (sp[1] << 8));
                 }
             }
@@ -229,8 +269,8 @@ void oracle_expert_lists(int T, int E, int k, const int32_t *idx, int32_t *offse
 static double oracle_silu(double g) { return g / (1.0 + exp(-g)); }
 
 /* SwiGLU expert on n tokens: out[t] = W_down (silu(W_gate x_t) * (W_up x_t)).
- * gate/up: [f x d], down: [d x f]; X, out: [n x d]. */
-void oracle_expert_ffn(int d, int f, int n, const double *X,
+ * gate/up: [f x d], down: [d x f]; X, out: [n x d]; codes of `bits` bits. */
+void oracle_expert_ffn(int d, int f, int n, int bits, const double *X,
                        const uint8_t *gc, const uint16_t *gs,
                        const uint8_t *uc, const uint16_t *us,
                        const uint8_t *dc, const uint16_t *ds, double *out)
@@ -239,9 +279,9 @@ void oracle_expert_ffn(int d, int f, int n, const double *X,
     double *Wu = (double *)malloc(sizeof(double) * (size_t)f * d);
     double *Wd = (double *)malloc(sizeof(double) * (size_t)d * f);
     double *h = (double *)malloc(sizeof(double) * (size_t)f);
-    oracle_dequant(f, d, gc, gs, Wg);
-    oracle_dequant(f, d, uc, us, Wu);
-    oracle_dequant(d, f, dc, ds, Wd);
+    oracle_dequant(f, d, bits, gc, gs, Wg);
+    oracle_dequant(f, d, bits, uc, us, Wu);
+    oracle_dequant(d, f, bits, dc, ds, Wd);
     for (int t = 0; t < n; ++t) {
         const double *x = X + (size_t)t * d;
         for (int r = 0; r < f; ++r) {
@@ -268,7 +308,7 @@ void oracle_expert_ffn(int d, int f, int n, const double *X,
 /* Whole layer for small shapes: route every token, run every selected
  * expert on its tokens, y[t] = sum_j w[t][j] * expert_{idx[t][j]}(x_t).
  * Expert e's weights are gc[e], gs[e], ... (pointer arrays of length E). */
-void oracle_moe_layer(int T, int d, int f, int E, int k, const uint16_t *x_bf16,
+void oracle_moe_layer(int T, int d, int f, int E, int k, int bits, const uint16_t *x_bf16,
                       const float *W, const float *bias,
                       const uint8_t *const *gc, const uint16_t *const *gs,
                       const uint8_t *const *uc, const uint16_t *const *us,
@@ -287,7 +327,7 @@ void oracle_moe_layer(int T, int d, int f, int E, int k, const uint16_t *x_bf16,
     for (int t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {
             int e = idx[(size_t)t * k + j];
-            oracle_expert_ffn(d, f, 1, X + (size_t)t * d, gc[e], gs[e], uc[e], us[e], dc[e], ds[e], o);
+            oracle_expert_ffn(d, f, 1, bits, X + (size_t)t * d, gc[e], gs[e], uc[e], us[e], dc[e], ds[e], o);
             for (int i = 0; i < d; ++i)
                 y[(size_t)t * d + i] += w[(size_t)t * k + j] * o[i];
         }

@@ -14,7 +14,8 @@ Generator (defined here; the device twin in ``synth_dev.cu`` restates it):
   Word ``i`` of a stream is ``mix64(key + (i + 1) * GAMMA)`` (mod 2**64), i.e.
   the SplitMix64 sequence started at ``key``.
 * Uniform codes: word ``i`` supplies codes ``32 i .. 32 i + 31`` as its 2-bit
-  fields, least significant first.
+  fields, least significant first; 4-bit codes: word ``i`` supplies codes
+  ``16 i .. 16 i + 15`` as its 4-bit fields.
 * Normals: Irwin-Hall with 12 terms. Normal ``i`` takes words ``4 i .. 4 i + 3``,
   each split into three 20-bit uniforms (bits 0-19, 20-39, 40-59); with ``S``
   the integer sum of the 12 fields, ``z = (S - 6 * 2**20) * 2**-20``. ``z`` is
@@ -102,6 +103,18 @@ def codes(key: int, n: int, start: int = 0) -> np.ndarray:
     return c[:n]
 
 
+def codes4(key: int, n: int, start: int = 0) -> np.ndarray:
+    """4-bit codes ``start .. start+n-1`` (uint8 in {0..15}); word ``i``
+    supplies codes ``16 i .. 16 i + 15`` as its 4-bit fields, least
+    significant first; ``start`` % 16 == 0."""
+    assert start % 16 == 0
+    nw = (n + 15) // 16
+    w = words(key, start // 16, nw)
+    sh = (np.arange(16, dtype=np.uint64) * np.uint64(4))[None, :]
+    c = ((w[:, None] >> sh) & np.uint64(15)).astype(np.uint8).reshape(-1)
+    return c[:n]
+
+
 def normals(key: int, n: int, start: int = 0) -> np.ndarray:
     """Irwin-Hall(12) normals ``start .. start+n-1`` as exact float32."""
     w = words(key, 4 * start, 4 * n).reshape(n, 4)
@@ -144,25 +157,31 @@ def gen_router_w(seed: int, layer: int, E: int, d: int) -> np.ndarray:
     return (np.float32(0.02) * z).astype(np.float32).reshape(E, d)
 
 
-def gen_codes(seed: int, layer: int, expert: int, mat: int, rows: int, K: int) -> np.ndarray:
-    """2-bit codes uint8 [rows, K] of one matrix of one expert."""
-    return codes(stream_key(seed, TAG_CODES, layer, expert, mat), rows * K).reshape(rows, K)
+def gen_codes(seed: int, layer: int, expert: int, mat: int, rows: int, K: int, bits: int = 2) -> np.ndarray:
+    """Codes uint8 [rows, K] of one matrix of one expert: 2-bit codes in
+    {0..3} or 4-bit codes in {0..15}."""
+    key = stream_key(seed, TAG_CODES, layer, expert, mat)
+    return (codes(key, rows * K) if bits == 2 else codes4(key, rows * K)).reshape(rows, K)
 
 
-def gen_scales(seed: int, layer: int, expert: int, mat: int, rows: int, K: int) -> np.ndarray:
-    """Block scales fp16(|N(0,0.02)| + 1e-3), float16 [rows, K/32]."""
+def gen_scales(seed: int, layer: int, expert: int, mat: int, rows: int, K: int, bits: int = 2) -> np.ndarray:
+    """Block scales, float16 [rows, K/32]: fp16(|N(0,0.02)| + 1e-3) for 2-bit
+    codes; for 4-bit codes the same value divided by 5, so that (c - 7.5) s
+    spans the range (c - 1.5) s does with 2-bit codes."""
     nb = rows * (K // 32)
     z = normals(stream_key(seed, TAG_SCALES, layer, expert, mat), nb)
     t = np.abs(np.float32(0.02) * z) + np.float32(1e-3)
+    if bits == 4:
+        t = t / np.float32(5.0)
     return t.astype(np.float32).astype(np.float16).reshape(rows, K // 32)
 
 
-def gen_expert(seed: int, layer: int, expert: int, d: int, f: int) -> dict:
+def gen_expert(seed: int, layer: int, expert: int, d: int, f: int, bits: int = 2) -> dict:
     """Codes and scales of one expert: gate/up [f, d], down [d, f]."""
-    out = {}
+    out = {"bits": bits}
     for name, mat, rows, K in (("gate", GATE, f, d), ("up", UP, f, d), ("down", DOWN, d, f)):
-        out[name + "_codes"] = gen_codes(seed, layer, expert, mat, rows, K)
-        out[name + "_scales"] = gen_scales(seed, layer, expert, mat, rows, K)
+        out[name + "_codes"] = gen_codes(seed, layer, expert, mat, rows, K, bits)
+        out[name + "_scales"] = gen_scales(seed, layer, expert, mat, rows, K, bits)
     return out
 
 
@@ -200,10 +219,11 @@ class Workload:
     zipf: bool
     seed: int
     chunk: int = 8192
+    bits: int = 2  # code width: 2 (Q2) or 4 (Q4)
 
     def desc(self) -> str:
         return (f"d={self.d} f={self.f} E={self.E} k={self.k} T={self.T} layers={self.layers} "
-                f"routing={'zipf1.1' if self.zipf else 'uniform'} seed={self.seed}")
+                f"routing={'zipf1.1' if self.zipf else 'uniform'} seed={self.seed} bits={self.bits}")
 
 
 WORKLOADS = {
@@ -219,6 +239,11 @@ WORKLOADS = {
     # the Coder variant of the model keeps 256 of the 512 experts per layer
     # ("Strata — 8~12GB 显存跑 125B 大模型的本地推理引擎", §5 models table)
     "coder_decode": Workload("coder_decode", 2048, 768, 256, 10, 1, 1, False, 5),
+    # the 4-bit block format (a wider level of the pages' quality ladder,
+    # "Strata：把 125B 大模型塞进 12GB 显卡…", 能跑多快 table)
+    "decode_q4": Workload("decode_q4", 2048, 768, 512, 10, 1, 1, False, 6, bits=4),
+    "verify4_q4": Workload("verify4_q4", 2048, 768, 512, 10, 4, 1, True, 6, bits=4),
+    "prefill_q4": Workload("prefill_q4", 2048, 768, 512, 10, 8192, 1, True, 6, bits=4),
 }
 
 

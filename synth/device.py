@@ -33,7 +33,8 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         V, I64 = ctypes.c_void_p, ctypes.c_int64
         lib.synth_codes.argtypes = [V, ctypes.c_int, I64, V, V]
-        lib.synth_scales.argtypes = [V, ctypes.c_int, I64, V, V]
+        lib.synth_codes4.argtypes = [V, ctypes.c_int, I64, V, V]
+        lib.synth_scales.argtypes = [V, ctypes.c_int, I64, ctypes.c_float, V, V]
         lib.synth_x_bf16.argtypes = [ctypes.c_uint64, I64, I64, V, V]
         lib.synth_router_w.argtypes = [ctypes.c_uint64, I64, V, V]
         for f in (lib.synth_codes, lib.synth_scales, lib.synth_x_bf16, lib.synth_router_w):
@@ -73,7 +74,7 @@ def _keys(seed, tag, layer, experts, mat):
     return torch.from_numpy(k.view(np.int64)).to("cuda")
 
 
-def expert_codes_scales(seed: int, layer: int, experts, mat: int, rows: int, K: int):
+def expert_codes_scales(seed: int, layer: int, experts, mat: int, rows: int, K: int, bits: int = 2):
     """codes uint8 [n, rows, K] and scales (fp16 bits as int16) [n, rows, K/32]."""
     import torch
     experts = list(experts)
@@ -82,8 +83,10 @@ def expert_codes_scales(seed: int, layer: int, experts, mat: int, rows: int, K: 
     scales = torch.empty((n, rows, K // 32), dtype=torch.int16, device="cuda")
     kc = _keys(seed, TAG_CODES, layer, experts, mat)
     ks = _keys(seed, TAG_SCALES, layer, experts, mat)
-    _chk(_load().synth_codes(kc.data_ptr(), n, rows * K, codes.data_ptr(), _stream()))
-    _chk(_load().synth_scales(ks.data_ptr(), n, rows * (K // 32), scales.data_ptr(), _stream()))
+    gen = _load().synth_codes if bits == 2 else _load().synth_codes4
+    _chk(gen(kc.data_ptr(), n, rows * K, codes.data_ptr(), _stream()))
+    _chk(_load().synth_scales(ks.data_ptr(), n, rows * (K // 32), ctypes.c_float(1.0 if bits == 2 else 5.0),
+                              scales.data_ptr(), _stream()))
     return codes, scales
 
 
@@ -94,14 +97,14 @@ def layer_blob(w: Workload, layer: int, pack_expert, out=None, batch: int = 32):
     library's device packer); this module only supplies the codes/scales."""
     import torch
     d, f, E = w.d, w.f, w.E
-    ebytes = 3 * d * f // 32 * 10
+    ebytes = 3 * (d // 64) * (f // 64) * (1280 if w.bits == 2 else 2304)
     if out is None:
         out = torch.empty(E * ebytes, dtype=torch.uint8, device="cuda")
     for e0 in range(0, E, batch):
         ex = list(range(e0, min(E, e0 + batch)))
-        gc, gs = expert_codes_scales(w.seed, layer, ex, GATE, f, d)
-        uc, us = expert_codes_scales(w.seed, layer, ex, UP, f, d)
-        dc, ds = expert_codes_scales(w.seed, layer, ex, DOWN, d, f)
+        gc, gs = expert_codes_scales(w.seed, layer, ex, GATE, f, d, w.bits)
+        uc, us = expert_codes_scales(w.seed, layer, ex, UP, f, d, w.bits)
+        dc, ds = expert_codes_scales(w.seed, layer, ex, DOWN, d, f, w.bits)
         for i, e in enumerate(ex):
             pack_expert(e, gc[i], gs[i], uc[i], us[i], dc[i], ds[i], out[e * ebytes:(e + 1) * ebytes])
     return out

@@ -3,7 +3,8 @@
 // It only draws inputs; it holds none of the layer's arithmetic.
 //
 // word(key, i) = mix64(key + (i + 1) * GAMMA), mix64 = SplitMix64 output
-// function. Codes: word i gives codes 32i..32i+31 (2-bit fields, LSB first).
+// function. Codes: word i gives codes 32i..32i+31 (2-bit fields, LSB first),
+// or 4-bit codes 16i..16i+15.
 // Normal i: Irwin-Hall over the 12 20-bit fields of words 4i..4i+3, exact
 // in float32; every later step is one IEEE round-to-nearest operation.
 #include <cuda_bf16.h>
@@ -50,13 +51,31 @@ __global__ void k_codes(const uint64_t *keys, int64_t n, uint8_t *out) {
     o[1] = make_uint4(b[4], b[5], b[6], b[7]);
 }
 
-// scales fp16(|0.02 z| + 1e-3)
-__global__ void k_scales(const uint64_t *keys, int64_t n, uint16_t *out) {
+// 4-bit codes: one thread per 16 codes (n % 16 == 0), word i -> codes 16i..16i+15
+__global__ void k_codes4(const uint64_t *keys, int64_t n, uint8_t *out) {
+    const int j = blockIdx.y;
+    const int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (w * 16 >= n) return;
+    const uint64_t v = word(keys[j], (uint64_t)w);
+    uint32_t b[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) x |= (uint32_t)((v >> (4 * (4 * q + r))) & 15u) << (8 * r);
+        b[q] = x;
+    }
+    *reinterpret_cast<uint4 *>(out + (size_t)j * n + (size_t)w * 16) = make_uint4(b[0], b[1], b[2], b[3]);
+}
+
+// scales fp16(|0.02 z| + 1e-3), divided by `div` (1 for 2-bit, 5 for 4-bit codes)
+__global__ void k_scales(const uint64_t *keys, int64_t n, float div, uint16_t *out) {
     const int j = blockIdx.y;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const float z = normal(keys[j], (uint64_t)i);
-    const float t = __fadd_rn(fabsf(__fmul_rn(0.02f, z)), 1e-3f);
+    float t = __fadd_rn(fabsf(__fmul_rn(0.02f, z)), 1e-3f);
+    if (div != 1.0f) t = __fdiv_rn(t, div);
     out[(size_t)j * n + i] = __half_as_ushort(__float2half_rn(t));
 }
 
@@ -83,9 +102,16 @@ int synth_codes(const uint64_t *keys_dev, int nkeys, int64_t n, uint8_t *out, cu
     return (int)cudaGetLastError();
 }
 
-int synth_scales(const uint64_t *keys_dev, int nkeys, int64_t n, uint16_t *out, cudaStream_t st) {
+int synth_codes4(const uint64_t *keys_dev, int nkeys, int64_t n, uint8_t *out, cudaStream_t st) {
+    if (n % 16) return -1;
+    dim3 grid((unsigned)((n / 16 + 255) / 256), nkeys);
+    k_codes4<<<grid, 256, 0, st>>>(keys_dev, n, out);
+    return (int)cudaGetLastError();
+}
+
+int synth_scales(const uint64_t *keys_dev, int nkeys, int64_t n, float div, uint16_t *out, cudaStream_t st) {
     dim3 grid((unsigned)((n + 255) / 256), nkeys);
-    k_scales<<<grid, 256, 0, st>>>(keys_dev, n, out);
+    k_scales<<<grid, 256, 0, st>>>(keys_dev, n, div, out);
     return (int)cudaGetLastError();
 }
 

@@ -43,10 +43,10 @@ def bf16_rne_exact(v: float) -> int:
     return int(np.array([r], dtype=np.float32).view(np.uint32)[0] >> 16)
 
 
-def load_tile_example():
-    blob = np.zeros(1280, dtype=np.uint8)
+def load_tile_example(name="q2_tile_example.txt", size=1280):
+    blob = np.zeros(size, dtype=np.uint8)
     expects = []
-    with open(os.path.join(GOLD, "q2_tile_example.txt")) as fh:
+    with open(os.path.join(GOLD, name)) as fh:
         for line in fh:
             t = line.split("#", 1)[0].split()
             if not t:
@@ -65,10 +65,10 @@ def load_tile_example():
     return blob, expects
 
 
-def const_expert(d, f, gate_code, up_code, down_code, scale=2.0):
+def const_expert(d, f, gate_code, up_code, down_code, scale=2.0, bits=2):
     """Expert whose three matrices hold one code everywhere, one scale."""
     s = np.float16(scale)
-    return dict(
+    return dict(bits=bits,
         gate_codes=np.full((f, d), gate_code, np.uint8), gate_scales=np.full((f, d // 32), s, np.float16),
         up_codes=np.full((f, d), up_code, np.uint8), up_scales=np.full((f, d // 32), s, np.float16),
         down_codes=np.full((d, f), down_code, np.uint8), down_scales=np.full((d, f // 32), s, np.float16))
@@ -90,10 +90,10 @@ def identity_like_expert(d, f, down_mult):
     return dict(gate_codes=gc, gate_scales=gs, up_codes=uc, up_scales=us, down_codes=dc, down_scales=ds)
 
 
-def tiny_layer(seed=0, T=8, d=256, f=128, E=16, k=4):
+def tiny_layer(seed=0, T=8, d=256, f=128, E=16, k=4, bits=2):
     x = synth.gen_x_bf16(seed, T, d)
     W = synth.gen_router_w(seed, 0, E, d)
-    experts = [synth.gen_expert(seed, 0, e, d, f) for e in range(E)]
+    experts = [synth.gen_expert(seed, 0, e, d, f, bits) for e in range(E)]
     return x, W, experts
 
 
@@ -160,6 +160,63 @@ def check_dequant_rules():
     assert np.array_equal(W[0, 32:], np.tile(base * 2.0, 8))
     assert np.array_equal(W[1, :32], np.tile(base * 1.0, 8))
     assert np.array_equal(W[1, 32:], np.tile(base * 0.5, 8))
+
+
+def check_q4_tile_example():
+    blob, expects = load_tile_example("q4_tile_example.txt", 2304)
+    codes, scales = O.unpack_q4_tiled(blob, 64, 64)
+    W = O.dequant(codes, scales, bits=4)
+    for r, c, code, val in expects:
+        assert codes[r, c] == code, f"4-bit code at ({r},{c}) = {codes[r, c]}, expected {code}"
+        assert W[r, c] == val, f"4-bit weight at ({r},{c}) = {W[r, c]}, expected {val}"
+    # row 0's codes are column % 16 everywhere; rows 2..62 all code 0 (-7.5)
+    assert np.array_equal(codes[0], np.arange(64) % 16)
+    assert np.all(W[2:63] == -7.5)
+
+
+def check_q4_dequant_rules():
+    # code c -> (c - 7.5) * s, one scale per 32 consecutive columns; codes c
+    # and 15 - c are exact negatives
+    codes = np.tile(np.arange(16, dtype=np.uint8), (2, 4))  # [2, 64]
+    scales = np.array([[0.25, 2.0], [1.0, 0.5]], dtype=np.float16)
+    W = O.dequant(codes, scales, bits=4)
+    base = np.arange(16) - 7.5
+    assert np.array_equal(W[0, :32], np.tile(base * 0.25, 2))
+    assert np.array_equal(W[0, 32:], np.tile(base * 2.0, 2))
+    assert np.array_equal(W[1, :32], np.tile(base * 1.0, 2))
+    assert np.array_equal(W[1, 32:], np.tile(base * 0.5, 2))
+    assert np.array_equal(W[:, :16], -W[:, 15::-1])
+
+
+def check_q4_swiglu_closed_form():
+    # gate code 9 (+1.5 s), up code 6 (-1.5 s), down code 8 (+0.5 s), scale 2:
+    # W_gate = +3, W_up = -3, W_down = +1; x = 1/32 everywhere -> g = 3, u = -3
+    d = f = 32
+    X = np.full((1, d), 1.0 / 32)
+    o = O.expert_ffn(X, const_expert(d, f, 9, 6, 8, bits=4))
+    ref = 1.0 * f * (silu_mp(3.0) * -3.0)
+    assert np.all(np.abs(o - ref) <= 1e-13 * abs(ref)), f"{o[0, 0]} vs {ref}"
+    # code 0 gate (-15), code 15 up (+15), code 1 down (-13), scale 2, d = 64
+    d, f = 64, 32
+    X = np.full((1, d), 1.0 / 64)
+    o = O.expert_ffn(X, const_expert(d, f, 0, 15, 1, bits=4))
+    ref = -13.0 * f * (silu_mp(-15.0) * 15.0)
+    assert np.all(np.abs(o - ref) <= 1e-13 * abs(ref)), f"{o[0, 0]} vs {ref}"
+
+
+def check_q4_dense_equals_sparse():
+    x, W, experts = tiny_layer(bits=4)
+    E, k = W.shape[0], 4
+    y, idx, w = O.moe_layer(x, W, None, experts, k)
+    X = synth.bf16_bits_to_f32(x).astype(np.float64)
+    gate = np.zeros((x.shape[0], E))
+    for t in range(x.shape[0]):
+        gate[t, idx[t]] = w[t]
+    dense = sum(gate[:, e:e + 1] * O.expert_ffn(X, experts[e]) for e in range(E))
+    assert rel(y, dense) <= 1e-12
+    # the same layer read as 2-bit codes would be a different layer
+    y2, _, _ = O.moe_layer(x, W, None, [dict(e, bits=2) for e in experts], k)
+    assert rel(y2, y) > 1e-3
 
 
 # ---------------------------------------------------------------- router

@@ -11,7 +11,16 @@ import oracle
 import pins_lib
 
 MUTANTS = [
-    ("code_offset", "W[(size_t)r * K + k] = (c - 1.5) * s;", "W[(size_t)r * K + k] = (c - 1.0) * s;"),
+    ("code_offset", "W[(size_t)r * K + k] = (c - offset) * s;", "W[(size_t)r * K + k] = (c - offset + 0.5) * s;"),
+    ("q4_offset", "double offset = ((double)(1 << bits) - 1.0) / 2.0;",
+     "double offset = bits == 4 ? 7.0 : ((double)(1 << bits) - 1.0) / 2.0;"),
+    ("q4_unpack_word", "const uint8_t *wp = tile + 32 * i + 4 * (2 * t + j / 2);",
+     "const uint8_t *wp = tile + 32 * i + 4 * (2 * t + j % 2);"),
+    ("q4_unpack_bit", "int bit = 16 * e + 8 * (j % 2) + 4 * sh;", "int bit = 16 * e + 4 * (j % 2) + 8 * sh;"),
+    ("q4_unpack_scales", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * b;", "const uint8_t *sp = tile + 2048 + 4 * i + 2 * (1 - b);"),
+    ("q4_code_mask", "codes[(size_t)r * K + 64 * s + c] = (uint8_t)((w >> bit) & 15u);",
+     "codes[(size_t)r * K + 64 * s + c] = (uint8_t)((w >> bit) & 7u);"),
+    ("expert_bits_ignored", "oracle_dequant(f, d, bits, uc, us, Wu);", "oracle_dequant(f, d, 2, uc, us, Wu);"),
     ("scale_block", "scales[(size_t)r * nb + k / 32]", "scales[(size_t)r * nb + k / 64]"),
     ("silu_sign", "g / (1.0 + exp(-g))", "g / (1.0 + exp(g))"),
     ("gate_up_swapped", "h[r] = oracle_silu(g) * u;", "h[r] = oracle_silu(u) * g;"),
