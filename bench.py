@@ -60,7 +60,8 @@ DECODE_KERNELS = 1
 
 # default timed steps per workload when --steps is not given
 DEFAULT_STEPS = {"decode": 64 * 1024, "verify4": 200, "verify6": 150, "verify16": 100, "prefill": 200,
-                 "prefill_stack": 3, "coder_decode": 64 * 1024}
+                 "prefill_stack": 3, "coder_decode": 64 * 1024,
+                 "decode_q4": 64 * 1024, "verify4_q4": 200, "prefill_q4": 200}
 
 
 def graph_steps(w) -> int:
@@ -205,8 +206,9 @@ class LayerData:
 
 
 def expert_bytes(w) -> int:
-    """Packed bytes of one expert: 3 matrices of d*f weights, 10 bytes per 32."""
-    return 3 * w.d * w.f // 32 * 10
+    """Packed bytes of one expert: 3 matrices of d*f weights, 10 bytes per 32
+    (2-bit codes + fp16 scale) or 18 (4-bit codes + fp16 scale)."""
+    return 3 * w.d * w.f // 32 * (10 if w.bits == 2 else 18)
 
 
 def decode_bytes(w, n_active):
@@ -238,19 +240,19 @@ class Runner:
         self.copies = copies_arg if self.rotate else (w.layers if self.stacked else 1)
         self.ntok = 64 if self.rotate else 1
         self.layer_gb = (w.E * expert_bytes(w) + w.E * w.d * 4) / 1e9
-        probe = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk)
+        probe = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk, bits=w.bits)
         self.layers = [LayerData(S, w, c, probe) for c in range(self.copies)]
         probe.close()
         T = w.T
         if self.stacked:
-            self.handle = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk)
+            self.handle = S.MoELayer(w.d, w.f, w.E, w.k, self.chunk, bits=w.bits)
             self.handles = []
             self.x0 = sd.x_bf16(w.seed, T, w.d, stream=rank).float()
             self.x_res = torch.empty((T, w.d), dtype=torch.float32, device=self.dev)
             self.xs = None
         else:
             self.handle = None
-            self.handles = [S.MoELayer(w.d, w.f, w.E, w.k, T, router_bias=self.layers[c].bias)
+            self.handles = [S.MoELayer(w.d, w.f, w.E, w.k, T, router_bias=self.layers[c].bias, bits=w.bits)
                             for c in range(self.copies)]
             self.xs = sd.x_bf16(w.seed, T * self.ntok, w.d, stream=rank).view(self.ntok, T, w.d)
             self.x_res = None
@@ -372,7 +374,7 @@ def stack_active_experts(run):
     xn = torch.empty((T, w.d), dtype=torch.bfloat16, device=run.dev)
     n_active = []
     for l in range(w.layers):
-        h = S.MoELayer(w.d, w.f, w.E, w.k, T, flags=S.STRATA_ACCUMULATE,
+        h = S.MoELayer(w.d, w.f, w.E, w.k, T, flags=S.STRATA_ACCUMULATE, bits=w.bits,
                        router_bias=run.layers[l].bias if w.zipf else None)
         S.strata_rmsnorm_bf16(x, xn, T, w.d, 1e-6)
         h.forward(xn, run.layers[l].W, run.layers[l].blob, x, T)
@@ -409,7 +411,7 @@ def prefill_roofline(w, dom_ms, layer_ms, peak, peak_src, peak_kind):
     ach = flops / (dom_ms * 1e-3) / 1e12
     layer = expert_flops(w, w.T) / (layer_ms * 1e-3) / 1e12
     traffic, tnote = measured_traffic("prefill") if w.name == "prefill" else (None, "no capture of this shape")
-    return {"bound": "tensor", "kernel": "k_expert_gemm<0> (gate/up + SwiGLU)", "achieved": ach, "peak": peak,
+    return {"bound": "tensor", "kernel": f"k_expert_gemm<0, {w.bits}> (gate/up + SwiGLU)", "achieved": ach, "peak": peak,
             "unit": "TFLOP/s", "frac": ach / peak, "traffic": traffic, "traffic_note": tnote,
             "algorithmic_flops_per_launch": flops, "avg_launch_ms": dom_ms,
             "avg_launch_ms_source": "CUDA events recorded by the library around the kernel, inside the graph",
@@ -548,7 +550,7 @@ def cpu_baseline(w, seconds):
 
     def src(e):
         if e not in src_cache:
-            src_cache[e] = synth.gen_expert(w.seed, 0, e, w.d, w.f)
+            src_cache[e] = synth.gen_expert(w.seed, 0, e, w.d, w.f, w.bits)
         return src_cache[e]
 
     if w.T <= 16:

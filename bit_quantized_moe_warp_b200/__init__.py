@@ -34,10 +34,13 @@ STRATA_ERR_TIMEOUT = -7
 STRATA_ERR_BOUNDS = -8
 
 STRATA_FMT_Q2_0_TILED = 1
+STRATA_FMT_Q4_0_TILED = 2
 STRATA_ACCUMULATE = 1
 STRATA_FORCE_PREFILL = 2
 STRATA_DECODE_MAX_TOKENS = 16
 STRATA_Q2_TILE_BYTES = 1280
+STRATA_Q4_TILE_BYTES = 2304
+FORMAT_OF_BITS = {2: STRATA_FMT_Q2_0_TILED, 4: STRATA_FMT_Q4_0_TILED}
 
 
 class strata_moe_desc(ctypes.Structure):
@@ -56,6 +59,7 @@ V, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
 DP = ctypes.POINTER(strata_moe_desc)
 _SIGS = {
     "strata_q2_matrix_bytes": (SZ, [I32, I32]),
+    "strata_q4_matrix_bytes": (SZ, [I32, I32]),
     "strata_moe_expert_bytes": (SZ, [DP]),
     "strata_moe_expert_blob_bytes": (SZ, [DP]),
     "strata_moe_workspace_bytes": (SZ, [DP]),
@@ -72,6 +76,7 @@ _SIGS = {
     "strata_moe_set_stage_events": (I32, [V, V, I32]),
     "strata_moe_check_status": (I32, [V]),
     "strata_q2_pack": (I32, [V, V, I32, I32, V]),
+    "strata_q4_pack": (I32, [V, V, I32, I32, V]),
     "strata_moe_pack_expert": (I32, [DP, V, V, V, V, V, V, V]),
     "strata_moe_pack_expert_device": (I32, [DP, V, V, V, V, V, V, V, V]),
     "strata_selftest_wait_timeout": (I32, [ctypes.c_uint64, V]),
@@ -110,8 +115,9 @@ def _check(status: int):
         raise StrataError(status, _lib.strata_last_error().decode(errors="replace"))
 
 
-def make_desc(d_model, d_ff, n_experts, top_k, max_tokens, flags=0, router_bias=None) -> strata_moe_desc:
-    return strata_moe_desc(d_model, d_ff, n_experts, top_k, max_tokens, 32, STRATA_FMT_Q2_0_TILED, flags,
+def make_desc(d_model, d_ff, n_experts, top_k, max_tokens, flags=0, router_bias=None, bits=2) -> strata_moe_desc:
+    """Layer descriptor; bits = 2 or 4 picks the weight format."""
+    return strata_moe_desc(d_model, d_ff, n_experts, top_k, max_tokens, 32, FORMAT_OF_BITS.get(bits, 0), flags,
                            _ptr(router_bias))
 
 
@@ -120,6 +126,10 @@ def make_desc(d_model, d_ff, n_experts, top_k, max_tokens, flags=0, router_bias=
 
 def strata_q2_matrix_bytes(rows, K):
     return _lib.strata_q2_matrix_bytes(rows, K)
+
+
+def strata_q4_matrix_bytes(rows, K):
+    return _lib.strata_q4_matrix_bytes(rows, K)
 
 
 def strata_moe_expert_bytes(desc):
@@ -216,6 +226,14 @@ def strata_q2_pack(codes, scales_fp16, rows, K, dst):
     _check(_lib.strata_q2_pack(c.ctypes.data, s.ctypes.data, rows, K, dst.ctypes.data))
 
 
+def strata_q4_pack(codes, scales_fp16, rows, K, dst):
+    """Host packer of the 4-bit format (codes 0..15), arguments as strata_q2_pack."""
+    import numpy as np
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(np.asarray(scales_fp16).view(np.uint16))
+    _check(_lib.strata_q4_pack(c.ctypes.data, s.ctypes.data, rows, K, dst.ctypes.data))
+
+
 def strata_moe_pack_expert(desc, gc, gs, uc, us, dc, ds, dst):
     """Host packer of one expert (numpy arrays)."""
     import numpy as np
@@ -256,9 +274,10 @@ def strata_last_error():
 class MoELayer:
     """Owns a layer handle (and keeps the desc's bias tensor alive)."""
 
-    def __init__(self, d_model, d_ff, n_experts, top_k, max_tokens, flags=0, router_bias=None, workspace=None):
+    def __init__(self, d_model, d_ff, n_experts, top_k, max_tokens, flags=0, router_bias=None, workspace=None,
+                 bits=2):
         self._bias = router_bias
-        self.desc = make_desc(d_model, d_ff, n_experts, top_k, max_tokens, flags, router_bias)
+        self.desc = make_desc(d_model, d_ff, n_experts, top_k, max_tokens, flags, router_bias, bits)
         nbytes = strata_moe_workspace_bytes(self.desc) if workspace is not None else 0
         self.handle = strata_moe_layer_create(self.desc, workspace, nbytes)
 

@@ -40,7 +40,9 @@
 // accumulates sum_k (base_k + c_k) x_k in fp32; subtracting the per-token
 // constant Z = sum_k base_k x_k + 1.5 sum_k x_k of each 32-column block and
 // multiplying by the block's fp16 scale gives sum_k (c_k - 1.5) s x_k, up to
-// fp32 rounding. Each token's x is staged as fp16(x * s) with s = 2^e putting
+// fp32 rounding. The 4-bit format (codes 0..15, offset 7.5) moves every
+// code to mantissa bits 4..7 (one shift per register at most), so all its
+// columns decode as 64 + c and Z = 71.5 sum_k x_k. Each token's x is staged as fp16(x * s) with s = 2^e putting
 // its largest |x| in [1, 2): exact for every element within 2^-14 of that
 // largest, whatever the token's magnitude; the router sums and the gate/up
 // dot products carry s and are divided by it exactly. h, which grows as x^2,
@@ -68,9 +70,16 @@ constexpr int kFusedMaxBuf = 16;
 // groups) per chunk, so the fixed cost of a chunk (all warps waking on its
 // barrier at once, loading the token fragments) is paid half as often as
 // with 20 KB chunks; measured on B200, 4% faster at 1 token, 2.5-4% at 4-16.
-constexpr int kGuSlicesPerChunk = 16;     // gate/up chunk: 16 K-slices x (gate, up) tiles = 40 KB
-constexpr int kDownPanelsPerChunk = 32;   // down chunk: 32 tiles of 64 d-rows = 40 KB
+// 4-bit tiles (2304 bytes) take 8 K-slices or 16 down tiles per chunk (36 KB).
 constexpr uint32_t kChunkBytes = 40960;
+template <int BITS>
+struct ChunkCfg {
+    static constexpr int kTile = Qn<BITS>::kTileBytes;
+    static constexpr int kGuSlices = BITS == 4 ? 8 : 16;     // gate/up chunk: K-slices x (gate, up) tiles
+    static constexpr int kDownPanels = BITS == 4 ? 16 : 32;  // down chunk: tiles of 64 d-rows
+    static_assert(kGuSlices * 2 * kTile <= (int)kChunkBytes && kDownPanels * kTile <= (int)kChunkBytes,
+                  "chunk exceeds a ring buffer");
+};
 constexpr int kHStride = 64 + 8;          // fp16 row stride of h (halves)
 constexpr int kRouterRowsMax = 16;        // router rows per CTA (E <= 16 * number of CTAs)
 // room left beside the dynamic shared memory for the kernel's static arrays
@@ -189,19 +198,71 @@ __host__ __device__ constexpr uint32_t step_magic(int j) {
 }
 __host__ __device__ constexpr float step_base(int j) { return j == 0 ? 16.f : j == 1 ? 64.f : j == 2 ? 256.f : 1024.f; }
 
-// The A-side words of one 16-row group of a tile: lane (g, t) reads word t
-// of rows g and g+8 and the two rows' block scales.
-struct TileRows {
+// The A-side words of one 16-row group of a tile: lane (g, t) reads, for
+// rows g and g+8, word t (2-bit) or words 2t, 2t+1 (4-bit), and the two
+// rows' block scales.
+template <int BITS>
+struct TileRows;
+template <>
+struct TileRows<2> {
     uint32_t wg, wg8, sg, sg8;
 };
-STRATA_DEV TileRows load_rows(const uint8_t *tile, int gr) {
+template <>
+struct TileRows<4> {
+    uint2 wg, wg8;
+    uint32_t sg, sg8;
+};
+template <int BITS>
+STRATA_DEV TileRows<BITS> load_rows(const uint8_t *tile, int gr) {
+    using F = Qn<BITS>;
     const int t = threadIdx.x & 3;
-    TileRows r;
-    r.wg = *reinterpret_cast<const uint32_t *>(tile + 16 * gr + 4 * t);
-    r.wg8 = *reinterpret_cast<const uint32_t *>(tile + 16 * (gr + 8) + 4 * t);
-    r.sg = *reinterpret_cast<const uint32_t *>(tile + kTileScaleOffset + 4 * gr);
-    r.sg8 = *reinterpret_cast<const uint32_t *>(tile + kTileScaleOffset + 4 * (gr + 8));
+    TileRows<BITS> r;
+    if constexpr (BITS == 4) {
+        r.wg = *reinterpret_cast<const uint2 *>(tile + F::kRowBytes * gr + 8 * t);
+        r.wg8 = *reinterpret_cast<const uint2 *>(tile + F::kRowBytes * (gr + 8) + 8 * t);
+    } else {
+        r.wg = *reinterpret_cast<const uint32_t *>(tile + F::kRowBytes * gr + 4 * t);
+        r.wg8 = *reinterpret_cast<const uint32_t *>(tile + F::kRowBytes * (gr + 8) + 4 * t);
+    }
+    r.sg = *reinterpret_cast<const uint32_t *>(tile + F::kScaleOffset + 4 * gr);
+    r.sg8 = *reinterpret_cast<const uint32_t *>(tile + F::kScaleOffset + 4 * (gr + 8));
     return r;
+}
+
+// A fragment of 16-column step j (registers: rows g / g+8 x columns 2t, 2t+1,
+// then 2t+8, 2t+9) as exact fp16 values base + code.
+// 2-bit: the step's codes sit at mantissa bit 6 - 2j of word t (base 16,
+// 64, 256, 1024); the second half (s = 1) is 8 bits higher.
+// 4-bit: word 2t + j/2, bits 8(j%2) + 4s: both halves are moved to bits
+// 4..7 (base 64).
+STRATA_DEV void a_frag(const TileRows<2> &w, int j, uint32_t (&a)[4]) {
+    const uint32_t m = 0x00030003u << (6 - 2 * j), g = step_magic(j);
+    a[0] = (w.wg & m) | g;
+    a[1] = (w.wg8 & m) | g;
+    a[2] = ((w.wg >> 8) & m) | g;
+    a[3] = ((w.wg8 >> 8) & m) | g;
+}
+STRATA_DEV void a_frag(const TileRows<4> &w, int j, uint32_t (&a)[4]) {
+    constexpr uint32_t m = 0x00F000F0u, g = 0x54005400u;
+    const uint32_t x = (j >> 1) ? w.wg.y : w.wg.x, x8 = (j >> 1) ? w.wg8.y : w.wg8.x;
+    if (j & 1) {
+        a[0] = ((x >> 4) & m) | g;
+        a[1] = ((x8 >> 4) & m) | g;
+        a[2] = ((x >> 8) & m) | g;
+        a[3] = ((x8 >> 8) & m) | g;
+    } else {
+        a[0] = ((x << 4) & m) | g;
+        a[1] = ((x8 << 4) & m) | g;
+        a[2] = (x & m) | g;
+        a[3] = (x8 & m) | g;
+    }
+}
+
+// block-constant weight of tile column 2l (and 2l+1): base of its step + the
+// format's code offset
+template <int BITS>
+STRATA_DEV float column_weight(int l) {
+    return BITS == 4 ? 71.5f : step_base(l >> 3) + 1.5f;
 }
 
 // One 16-row group x one 64-column tile x NT n-tiles of 8 token slots.
@@ -211,9 +272,8 @@ STRATA_DEV TileRows load_rows(const uint8_t *tile, int gr) {
 // ODD false (one token: only slot 0 is real) the odd slots are left alone.
 // NT is the number of n-tiles that hold tokens: no per-tile predicate sits
 // between the MMAs (it costs about half the loop's throughput).
-template <int NT, bool ODD, typename BSrc, typename ZSrc>
-STRATA_DEV void tile_mma(const TileRows &w, BSrc bsrc, ZSrc zsrc, float (&out)[NT][4]) {
-    const uint32_t v8g = w.wg >> 8, v8g8 = w.wg8 >> 8;
+template <int NT, bool ODD, int BITS, typename BSrc, typename ZSrc>
+STRATA_DEV void tile_mma(const TileRows<BITS> &w, BSrc bsrc, ZSrc zsrc, float (&out)[NT][4]) {
     const float2 s_g = __half22float2(*reinterpret_cast<const __half2 *>(&w.sg));
     const float2 s_g8 = __half22float2(*reinterpret_cast<const __half2 *>(&w.sg8));
 #pragma unroll
@@ -226,8 +286,8 @@ STRATA_DEV void tile_mma(const TileRows &w, BSrc bsrc, ZSrc zsrc, float (&out)[N
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
             const int j = 2 * blk + jj;
-            const uint32_t m = 0x00030003u << (6 - 2 * j), g = step_magic(j);
-            const uint32_t a[4] = {(w.wg & m) | g, (w.wg8 & m) | g, (v8g & m) | g, (v8g8 & m) | g};
+            uint32_t a[4];
+            a_frag(w, j, a);
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 uint32_t b0, b1;
@@ -251,14 +311,15 @@ STRATA_DEV void tile_mma(const TileRows &w, BSrc bsrc, ZSrc zsrc, float (&out)[N
 }
 
 // Per-block constants of one staged fp16 row (columns in 64-column tiles),
-// one warp: z[b] = sum over the block's columns k of (base_j(k) + 1.5) x_k,
-// i.e. sum_j base_j X_j + 1.5 X_b. Lane l reads columns 2l, 2l+1 of each
-// tile (step j = l / 8, block l / 16) and the 16 lanes of a block reduce by
-// shuffles, so the reads are conflict-free; four tiles at a time keep four
-// independent shuffle chains in flight.
+// one warp: z[b] = sum over the block's columns k of (base(k) + offset) x_k
+// (2-bit: sum_j base_j X_j + 1.5 X_b; 4-bit: 71.5 X_b). Lane l reads
+// columns 2l, 2l+1 of each tile (step j = l / 8, block l / 16) and the 16
+// lanes of a block reduce by shuffles, so the reads are conflict-free; four
+// tiles at a time keep four independent shuffle chains in flight.
+template <int BITS>
 STRATA_DEV void row_block_constants(const __half *row, int ncols, float *z) {
     const int lane = threadIdx.x & 31;
-    const float wgt = step_base(lane >> 3) + 1.5f;
+    const float wgt = column_weight<BITS>(lane);
     for (int c0 = 0; c0 < ncols; c0 += 256) {
         float sum[4];
 #pragma unroll
@@ -282,7 +343,7 @@ STRATA_DEV void row_block_constants(const __half *row, int ncols, float *z) {
 
 // One gate/up K slice for the warp's RGM (matrix, row group) pairs: the
 // slice's token fragments are loaded once and reused for every pair.
-template <int NTA, int NT, int RGM, bool ODD>
+template <int NTA, int NT, int RGM, bool ODD, int BITS>
 STRATA_DEV void gu_slice(const uint8_t *tiles, const __half *const (&xb)[NT], const float *const (&z0)[NT],
                          const float *const (&z1)[NT], int col0, int rgm0, int g, float (&out)[RGM][NT][4]) {
     uint32_t bf[NTA][4][2];
@@ -300,7 +361,7 @@ STRATA_DEV void gu_slice(const uint8_t *tiles, const __half *const (&xb)[NT], co
 #pragma unroll
     for (int r = 0; r < RGM; ++r) {
         const int rgm = rgm0 + r, m = rgm >> 2, gr = 16 * (rgm & 3) + g;
-        const TileRows w = load_rows(tiles + m * kTileBytes, gr);
+        const TileRows<BITS> w = load_rows<BITS>(tiles + m * Qn<BITS>::kTileBytes, gr);
         tile_mma<NTA, ODD>(
             w,
             [&](int n, int j, uint32_t &b0, uint32_t &b1) {
@@ -317,8 +378,8 @@ STRATA_DEV void gu_slice(const uint8_t *tiles, const __half *const (&xb)[NT], co
 
 // One down tile row group with h fragments and block constants held in
 // registers for the whole unit.
-template <int NTA, int NT, bool ODD>
-STRATA_DEV void down_rows(const TileRows &w, const uint32_t (&bf)[NT][4][2], const float (&zf)[NT][2][2],
+template <int NTA, int NT, bool ODD, int BITS>
+STRATA_DEV void down_rows(const TileRows<BITS> &w, const uint32_t (&bf)[NT][4][2], const float (&zf)[NT][2][2],
                           float (&o)[NT][4]) {
     tile_mma<NTA, ODD>(
         w,
@@ -333,8 +394,9 @@ STRATA_DEV void down_rows(const TileRows &w, const uint32_t (&bf)[NT][4][2], con
         reinterpret_cast<float(&)[NTA][4]>(o));
 }
 
-template <int TT>
+template <int TT, int BITS>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedArgs a) {
+    using CC = ChunkCfg<BITS>;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar;
     __shared__ int s_abort;
@@ -561,11 +623,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             for (int j = lane; j < k; j += 32) sel_w[warp * k + j] = expf(sel_val[warp * k + j] - vmax) / den;
         } else {  // warps without a token meanwhile compute the per-block constants of x (used in phase 2)
             for (int r = warp - T; r < T; r += kFusedComputeWarps - T)
-                row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
+                row_block_constants<BITS>(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         }
         if (T >= kFusedComputeWarps)  // no warp was free
             for (int r = warp; r < T; r += kFusedComputeWarps)
-                row_block_constants(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
+                row_block_constants<BITS>(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         compute_sync();
         for (int i = tid; i < T * k; i += 512)
             if (in_bounds(sel_idx[i], E, status)) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
@@ -654,8 +716,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     // ---------------------------------------------------------------- phase 2
     const int FP = f / 64;   // 64-row slices of the hidden layer
     const int SLK = d / 64;  // K slices of gate/up = 64-row panels of down
-    const int nG = (SLK + kGuSlicesPerChunk - 1) / kGuSlicesPerChunk;
-    const int nD = (SLK + kDownPanelsPerChunk - 1) / kDownPanelsPerChunk;
+    const int nG = (SLK + CC::kGuSlices - 1) / CC::kGuSlices;
+    const int nD = (SLK + CC::kDownPanels - 1) / CC::kDownPanels;
     const int n_units = n_act * FP;
     const int nq = (n_units > b) ? (n_units - b + G - 1) / G : 0;
     // chunk i of unit u: its source and size
@@ -663,12 +725,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         const uint8_t *ebase = a.blob + (size_t)checked_index(act[u / FP], E, 0, status) * a.ebytes;
         const int p = u % FP;
         if (i < nG) {
-            const int s0 = i * kGuSlicesPerChunk, ns = min(kGuSlicesPerChunk, SLK - s0);
-            bytes = (uint32_t)ns * 2u * kTileBytes;
+            const int s0 = i * CC::kGuSlices, ns = min(CC::kGuSlices, SLK - s0);
+            bytes = (uint32_t)ns * 2u * CC::kTile;
             return ebase + (size_t)p * a.xs.gu_panel + (size_t)s0 * a.xs.gu_slice;
         }
-        const int p0 = (i - nG) * kDownPanelsPerChunk, np = min(kDownPanelsPerChunk, SLK - p0);
-        bytes = (uint32_t)np * kTileBytes;
+        const int p0 = (i - nG) * CC::kDownPanels, np = min(CC::kDownPanels, SLK - p0);
+        bytes = (uint32_t)np * CC::kTile;
         return ebase + a.down_off + (size_t)p * a.xs.dn_slice + (size_t)p0 * a.xs.dn_panel;
     };
 
@@ -755,14 +817,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     if (!bad) bad = !mbar_wait(&full[bi], (uint32_t)((c / a.nbuf) & 1), status, &s_abort);
                     if (!bad) {
                         const uint8_t *buf = bufs + (size_t)bi * kChunkBytes;
-                        const int s0 = i * kGuSlicesPerChunk, ns = min(kGuSlicesPerChunk, SLK - s0);
+                        const int s0 = i * CC::kGuSlices, ns = min(CC::kGuSlices, SLK - s0);
                         for (int sl = kq; sl < ns; sl += KSPLIT) {
-                            const uint8_t *tiles = buf + (size_t)sl * 2 * kTileBytes;
+                            const uint8_t *tiles = buf + (size_t)sl * 2 * CC::kTile;
                             const int col0 = (s0 + sl) * 64;
                             if (NT == 1 || nta == 1)
-                                gu_slice<1, NT, RGM, ODD>(tiles, xb, z0, z1, col0, rgm0, g, out);
+                                gu_slice<1, NT, RGM, ODD, BITS>(tiles, xb, z0, z1, col0, rgm0, g, out);
                             else
-                                gu_slice<NT, NT, RGM, ODD>(tiles, xb, z0, z1, col0, rgm0, g, out);
+                                gu_slice<NT, NT, RGM, ODD, BITS>(tiles, xb, z0, z1, col0, rgm0, g, out);
                         }
                     }
                     __syncwarp();
@@ -811,7 +873,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 hh[slot * kHStride + row] = __float2half_rn(h);
             }
             compute_sync();
-            if (warp < NS) row_block_constants(hh + warp * kHStride, 64, hz + warp * 2);
+            if (warp < NS) row_block_constants<BITS>(hh + warp * kHStride, 64, hz + warp * 2);
             compute_sync();
             // ---- down: y[token] += w * W_down[:, slice] h
             {
@@ -844,19 +906,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     if (!bad) bad = !mbar_wait(&full[bi], (uint32_t)((c / a.nbuf) & 1), status, &s_abort);
                     if (!bad) {
                         const uint8_t *buf = bufs + (size_t)bi * kChunkBytes;
-                        const int p0 = i * kDownPanelsPerChunk, np = min(kDownPanelsPerChunk, SLK - p0);
+                        const int p0 = i * CC::kDownPanels, np = min(CC::kDownPanels, SLK - p0);
                         for (int rgi = warp; rgi < np * 4; rgi += kFusedComputeWarps) {
                             const int pan = rgi >> 2, r16 = 16 * (rgi & 3) + g;
-                            const TileRows w = load_rows(buf + (size_t)pan * kTileBytes, r16);
+                            const TileRows<BITS> w = load_rows<BITS>(buf + (size_t)pan * CC::kTile, r16);
                             float o[NT][4];
 #pragma unroll
                             for (int n = 0; n < NT; ++n)
 #pragma unroll
                                 for (int z = 0; z < 4; ++z) o[n][z] = 0.f;
                             if (NT == 1 || nta == 1)
-                                down_rows<1, NT, ODD>(w, bf, zf, o);
+                                down_rows<1, NT, ODD, BITS>(w, bf, zf, o);
                             else
-                                down_rows<NT, NT, ODD>(w, bf, zf, o);
+                                down_rows<NT, NT, ODD, BITS>(w, bf, zf, o);
                             const int row = (p0 + pan) * 64 + r16;
 #pragma unroll
                             for (int n = 0; n < NT; ++n) {
@@ -942,7 +1004,15 @@ bool decode_fused_supported(const Shape &s, int T, int max_smem, int num_sms) {
 // (less L1), which slows the MMA loops (see kFusedSmemSoftCap). Kept per
 // device and instantiation; raised at layer creation, before any capture.
 static std::mutex g_limit_mutex;
-static int g_limit[64][3];
+static int g_limit[64][6];
+
+// the instantiation of a token count and code width
+using FusedKernel = void (*)(const FusedArgs);
+static FusedKernel kernel_of(int slot) {
+    static const FusedKernel k[6] = {k_decode_fused<1, 2>, k_decode_fused<4, 2>, k_decode_fused<16, 2>,
+                                     k_decode_fused<1, 4>, k_decode_fused<4, 4>, k_decode_fused<16, 4>};
+    return k[slot];
+}
 
 static cudaError_t ensure_limit(int slot, int need) {
     int dev = 0;
@@ -951,21 +1021,19 @@ static cudaError_t ensure_limit(int slot, int need) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_limit_mutex);
     if (g_limit[dev][slot] >= need) return cudaSuccess;
-    if (slot == 0) e = cudaFuncSetAttribute(k_decode_fused<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
-    if (slot == 1) e = cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
-    if (slot == 2) e = cudaFuncSetAttribute(k_decode_fused<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+    e = cudaFuncSetAttribute(kernel_of(slot), cudaFuncAttributeMaxDynamicSharedMemorySize, need);
     if (e == cudaSuccess) g_limit[dev][slot] = need;
     return e;
 }
 
-static int slot_of(int T) { return T <= 1 ? 0 : T <= 4 ? 1 : 2; }
+static int slot_of(int T, int bits) { return (T <= 1 ? 0 : T <= 4 ? 1 : 2) + (bits == 4 ? 3 : 0); }
 
 cudaError_t init_fused_attributes(const Shape &s, int max_tokens, int max_smem, int num_sms) {
     static const int tts[3] = {1, 4, 16};
     for (int i = 0; i < 3; ++i) {
         const int T = tts[i] < max_tokens ? tts[i] : max_tokens;
-        if (slot_of(T) != i || !decode_fused_supported(s, T, max_smem, num_sms)) continue;
-        const cudaError_t e = ensure_limit(i, (int)fused_config(s, T, max_smem).smem);
+        if (slot_of(T, 2) != i || !decode_fused_supported(s, T, max_smem, num_sms)) continue;
+        const cudaError_t e = ensure_limit(slot_of(T, s.bits), (int)fused_config(s, T, max_smem).smem);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -1004,15 +1072,11 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = ensure_limit(slot_of(T), (int)c.smem);  // a no-op after layer creation
+    const int slot = slot_of(T, s.bits);
+    cudaError_t e = ensure_limit(slot, (int)c.smem);  // a no-op after layer creation
     if (e != cudaSuccess) return e;
     if (ev) cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal);
-    if (T <= 1)
-        e = cudaLaunchKernelEx(&cfg, k_decode_fused<1>, a);
-    else if (T <= 4)
-        e = cudaLaunchKernelEx(&cfg, k_decode_fused<4>, a);
-    else
-        e = cudaLaunchKernelEx(&cfg, k_decode_fused<16>, a);
+    e = cudaLaunchKernelEx(&cfg, kernel_of(slot), a);
     if (ev) cudaEventRecordWithFlags(ev[3], st, cudaEventRecordExternal);
     return e;
 }

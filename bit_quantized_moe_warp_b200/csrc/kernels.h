@@ -46,6 +46,7 @@ constexpr int kGemm2N = 256;          // down GEMM: max tokens per tile
 
 struct Shape {
     int d, f, E, k;
+    int bits;  // code width of the expert weights: 2 or 4
 };
 
 struct TmaMaps {
@@ -89,7 +90,7 @@ void launch_combine(const Workspace &ws, float *y, bool accumulate, int T, const
 
 // --- misc
 void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cudaStream_t st);
-void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
+void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, int bits, uint8_t *dst,
                                size_t panel_stride, size_t slice_stride, cudaStream_t st);
 void launch_wait_selftest(uint32_t *status, uint64_t timeout_ns, cudaStream_t st);
 // one index one past the end of a 16-entry array, tested with in_bounds (the
@@ -98,20 +99,28 @@ void launch_bounds_selftest(uint32_t *status, cudaStream_t st);
 
 size_t expert_bytes(const Shape &s);
 
-// Q2 tiles: 64 rows x 64 columns, codes then scales.
+// Tiles: 64 rows x 64 columns, codes then scales. 2-bit: 16 code bytes per
+// row; 4-bit: 32. Qn<BITS> gives a format's sizes at compile time.
 constexpr int kTileRows = 64;
-constexpr int kTileBytes = 1280;
-constexpr int kTileScaleOffset = 1024;
+template <int BITS>
+struct Qn {
+    static constexpr int kRowBytes = 64 * BITS / 8;                // code bytes of one tile row
+    static constexpr int kScaleOffset = 64 * kRowBytes;            // 1024 or 2048
+    static constexpr int kTileBytes = kScaleOffset + 64 * 4;       // 1280 or 2304
+};
+constexpr int kTileBytes = Qn<2>::kTileBytes;
+constexpr int kTileScaleOffset = Qn<2>::kScaleOffset;
+inline size_t tile_bytes(const Shape &s) { return s.bits == 4 ? Qn<4>::kTileBytes : Qn<2>::kTileBytes; }
 
 // Byte strides between the tiles of an expert's matrices: gate/up tiles
-// (f-panel p, d-slice s) at p * gu_panel + s * gu_slice (gate, then up at
-// +1280); down tiles (d-panel p, f-slice s) at p * dn_panel + s * dn_slice.
+// (f-panel p, d-slice s) at p * gu_panel + s * gu_slice (gate, then up one
+// tile later); down tiles (d-panel p, f-slice s) at p * dn_panel + s * dn_slice.
 struct ExpertStrides {
     size_t gu_panel, gu_slice, dn_panel, dn_slice;
 };
 inline ExpertStrides expert_strides(const Shape &s) {
-    return ExpertStrides{(size_t)(s.d / 64) * 2 * kTileBytes, (size_t)2 * kTileBytes, (size_t)kTileBytes,
-                         (size_t)(s.d / 64) * kTileBytes};
+    const size_t tb = tile_bytes(s);
+    return ExpertStrides{(size_t)(s.d / 64) * 2 * tb, 2 * tb, tb, (size_t)(s.d / 64) * tb};
 }
 
 size_t down_section_offset(const Shape &s);

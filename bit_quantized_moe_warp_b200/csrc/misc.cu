@@ -34,11 +34,15 @@ void launch_rmsnorm_bf16(const float *x, void *out, int T, int d, float eps, cud
 }
 
 // ------------------------------------------------------------ packer
-// One thread per (tile, row): 64 codes -> four words (column
-// c = 16j + 8s + 2t + h in word t at bit 16h + 8s + 6 - 2j), then the row's
-// two block scales. Tile (p, s) goes to dst + p * panel_stride + s * slice_stride.
+// One thread per (tile, row): 64 codes -> the row's code words, then its two
+// block scales. Column c = 16j + 8s + 2t + h: 2-bit, word t at bit
+// 16h + 8s + 6 - 2j (four words); 4-bit, word 2t + j/2 at bit
+// 16h + 8(j%2) + 4s (eight words). Tile (p, s) goes to
+// dst + p * panel_stride + s * slice_stride.
+template <int BITS>
 __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales, int rows, int K,
                               uint8_t *__restrict__ dst, size_t panel_stride, size_t slice_stride) {
+    using F = Qn<BITS>;
     const int slices = K / 64;
     const long long n = (long long)(rows / kTileRows) * slices * kTileRows;
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -48,24 +52,32 @@ __global__ void k_pack_matrix(const uint8_t *__restrict__ codes, const uint16_t 
     const int p = (int)(tile / slices), s = (int)(tile % slices);
     const int r = p * kTileRows + i;
     const uint8_t *cr = codes + (size_t)r * K + (size_t)s * 64;
-    uint32_t w[4] = {0, 0, 0, 0};
+    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll 4
     for (int c = 0; c < 64; ++c) {
-        const uint32_t v = cr[c] & 3u;
-        w[(c & 7) >> 1] |= v << (16 * (c & 1) + 8 * ((c >> 3) & 1) + 6 - 2 * (c >> 4));
+        const int j = c >> 4, sh = (c >> 3) & 1, tq = (c & 7) >> 1, h = c & 1;
+        if (BITS == 4)
+            w[2 * tq + (j >> 1)] |= (cr[c] & 15u) << (16 * h + 8 * (j & 1) + 4 * sh);
+        else
+            w[tq] |= (cr[c] & 3u) << (16 * h + 8 * sh + 6 - 2 * j);
     }
     uint8_t *t = dst + (size_t)p * panel_stride + (size_t)s * slice_stride;
-    *reinterpret_cast<uint4 *>(t + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+    uint4 *tw = reinterpret_cast<uint4 *>(t + F::kRowBytes * i);
+    tw[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (BITS == 4) tw[1] = make_uint4(w[4], w[5], w[6], w[7]);
     const uint16_t *sr = scales + (size_t)r * (K / 32) + 2 * s;
-    *reinterpret_cast<uint32_t *>(t + kTileScaleOffset + 4 * i) = (uint32_t)sr[0] | ((uint32_t)sr[1] << 16);
+    *reinterpret_cast<uint32_t *>(t + F::kScaleOffset + 4 * i) = (uint32_t)sr[0] | ((uint32_t)sr[1] << 16);
 }
 
-void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
+void launch_pack_matrix_device(const uint8_t *codes, const uint16_t *scales, int rows, int K, int bits, uint8_t *dst,
                                size_t panel_stride, size_t slice_stride, cudaStream_t st) {
     const long long n = (long long)(rows / kTileRows) * (K / 64) * kTileRows;
     if (n <= 0) return;
-    k_pack_matrix<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(codes, scales, rows, K, dst, panel_stride,
-                                                                slice_stride);
+    const unsigned grid = (unsigned)((n + 255) / 256);
+    if (bits == 4)
+        k_pack_matrix<4><<<grid, 256, 0, st>>>(codes, scales, rows, K, dst, panel_stride, slice_stride);
+    else
+        k_pack_matrix<2><<<grid, 256, 0, st>>>(codes, scales, rows, K, dst, panel_stride, slice_stride);
 }
 
 // ------------------------------------------------------------ self test

@@ -1,5 +1,6 @@
 // prefill_gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores
-// (tcgen05, accumulators in tensor memory) for prefill chunks.
+// (tcgen05, accumulators in tensor memory) for prefill chunks, on 2-bit or
+// 4-bit tiles.
 //
 // Prompts are read in chunks of up to 8,192 tokens and the expert products
 // run on the quantised weights instead of first expanding them to FP16 in
@@ -26,26 +27,30 @@
 
 namespace strata {
 
-template <int MODE>
+// Stages: four, except gate/up on 4-bit tiles, whose four stages (57 KB
+// each) would not fit in 227 KB of shared memory.
+template <int MODE, int BITS>
 struct GCfg;
-template <>
-struct GCfg<0> {
-    static constexpr int NMAT = 2, NMAX = kGemm1N, STAGES = 4;
+template <int BITS>
+struct GCfg<0, BITS> {
+    static constexpr int NMAT = 2, NMAX = kGemm1N, STAGES = BITS == 4 ? 3 : 4;
 };
-template <>
-struct GCfg<1> {
+template <int BITS>
+struct GCfg<1, BITS> {
     static constexpr int NMAT = 1, NMAX = kGemm2N, STAGES = 4;
 };
 
 constexpr int kGemmThreads = 448;
 constexpr int kDequantWarps = 8;
 
-template <int MODE>
+template <int MODE, int BITS>
 struct GLayout {
-    static constexpr int NMAT = GCfg<MODE>::NMAT, NMAX = GCfg<MODE>::NMAX, STAGES = GCfg<MODE>::STAGES;
+    static constexpr int NMAT = GCfg<MODE, BITS>::NMAT, NMAX = GCfg<MODE, BITS>::NMAX,
+                         STAGES = GCfg<MODE, BITS>::STAGES;
+    static constexpr uint32_t TILE = Qn<BITS>::kTileBytes;
     static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // one fp16 matrix tile
     static constexpr uint32_t B_BYTES = NMAX * 128;    // NMAX rows of 64 fp16
-    static constexpr uint32_t W_BYTES = NMAT * 2 * kTileBytes;  // packed 2-bit tiles: 128 rows per matrix
+    static constexpr uint32_t W_BYTES = NMAT * 2 * TILE;  // packed tiles: 128 rows per matrix
     static constexpr uint32_t STAGE = ((NMAT * A_BYTES + B_BYTES + W_BYTES) + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM = STAGES * STAGE + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -82,9 +87,89 @@ STRATA_DEV int4 tile_at(const GemmArgs &a, int i) {
     return tl;
 }
 
-template <int MODE>
+// One row of a 64 x 64 2-bit tile -> fp16 (c - 1.5) s into output chunks
+// c_lo..c_hi-1 (columns 8c..8c+7) of a 128-byte swizzled A row.
+STRATA_DEV void dequant_row_q2(const uint8_t *wt, int ri, int c_lo, int c_hi, int row, uint8_t *arow) {
+    using F = Qn<2>;
+    const uint4 cw = *reinterpret_cast<const uint4 *>(wt + F::kRowBytes * ri);
+    uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + F::kScaleOffset + 4 * ri);
+    const __half2 s01 = *reinterpret_cast<__half2 *>(&scb);
+    const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+    const uint32_t words8[4] = {cw.x >> 8, cw.y >> 8, cw.z >> 8, cw.w >> 8};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // output chunk c: columns 8c .. 8c+7
+        if (c < c_lo || c >= c_hi) continue;
+        const __half2 sc = (c < 4) ? sh0 : sh1;
+        // Columns 8c + 2t, 8c + 2t + 1 (step j = c / 2, half s = c % 2)
+        // sit in word t at bits 8s + 6 - 2j and 16 + 8s + 6 - 2j. With
+        // the exponent that gives bit 6 - 2j the place value 1, the
+        // masked pair reads as the exact fp16 values base_j + code
+        // (base 16, 64, 256, 1024); subtracting base_j + 1.5 is exact
+        // for j < 3 (17.5, 65.5, 257.5), and in two exact steps for
+        // j = 3; one multiply by the scale rounds once.
+        const int j = c >> 1;
+        const uint32_t m = 0x00030003u << (6 - 2 * j);
+        const uint32_t g = j == 0 ? 0x4C004C00u : j == 1 ? 0x54005400u : j == 2 ? 0x5C005C00u : 0x64006400u;
+        uint32_t out[4];
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+            uint32_t v = (((c & 1) ? words8[pr] : words[pr]) & m) | g;
+            __half2 h = *reinterpret_cast<__half2 *>(&v);
+            if (j < 3) {
+                const float off = j == 0 ? 17.5f : j == 1 ? 65.5f : 257.5f;
+                h = __hsub2(h, __floats2half2_rn(off, off));
+            } else {
+                h = __hsub2(__hsub2(h, __floats2half2_rn(1024.f, 1024.f)), __floats2half2_rn(1.5f, 1.5f));
+            }
+            h = __hmul2(h, sc);  // (c - 1.5) s
+            out[pr] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// The same for a 4-bit tile row: (c - 7.5) s. Column 8c + 2t + h (chunk
+// c = 2j + s) sits in word 2t + j/2 at bits 16h + 8(j%2) + 4s; every pair is
+// moved to bits 4..7 / 20..23, where the exponent of 64 gives bit 4 the place
+// value 1, so it reads as 64 + code; subtracting 71.5 is exact, and one
+// multiply by the scale rounds once.
+STRATA_DEV void dequant_row_q4(const uint8_t *wt, int ri, int c_lo, int c_hi, int row, uint8_t *arow) {
+    using F = Qn<4>;
+    // the row's 32 code bytes as two 16-byte loads; rows 4..7 of each group
+    // of 8 take the halves in the other order, so 8 lanes hit 32 banks
+    const int sw = (ri >> 2) & 1;
+    const uint4 q0 = *reinterpret_cast<const uint4 *>(wt + F::kRowBytes * ri + 16 * sw);
+    const uint4 q1 = *reinterpret_cast<const uint4 *>(wt + F::kRowBytes * ri + 16 * (sw ^ 1));
+    const uint4 lo = sw ? q1 : q0, hi = sw ? q0 : q1;
+    const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + F::kScaleOffset + 4 * ri);
+    const __half2 s01 = *reinterpret_cast<__half2 *>(&scb);
+    const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
+    const __half2 off = __floats2half2_rn(71.5f, 71.5f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        if (c < c_lo || c >= c_hi) continue;
+        const __half2 sc = (c < 4) ? sh0 : sh1;
+        const int j = c >> 1, sh = 8 * (j & 1) + 4 * (c & 1);  // bit of the pair's low code
+        uint32_t out[4];
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+            const uint32_t w = words[2 * pr + (j >> 1)];
+            const uint32_t at4 = sh >= 4 ? (w >> (sh - 4)) : (w << 4);
+            uint32_t v = (at4 & 0x00F000F0u) | 0x54005400u;
+            __half2 h = __hsub2(*reinterpret_cast<__half2 *>(&v), off);
+            h = __hmul2(h, sc);  // (c - 7.5) s
+            out[pr] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_constant__ TmaMaps maps, GemmArgs a) {
-    using L = GLayout<MODE>;
+    using L = GLayout<MODE, BITS>;
+    constexpr uint32_t TB = L::TILE;
     constexpr int NMAT = L::NMAT, NMAX = L::NMAX, S = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -146,11 +231,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     }
                     mbar_arrive_expect_tx(&full[st], L::W_BYTES + brows * 128);
                     if (MODE == 0) {  // (gate, up) pairs of the panel's two 64-row halves
-                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * kTileBytes, &full[st]);
-                        bulk_g2s(W_at(st) + 2 * kTileBytes, wsrc + a.tile_panel + (size_t)ks * a.tile_slice,
-                                 2 * kTileBytes, &full[st]);
+                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * TB, &full[st]);
+                        bulk_g2s(W_at(st) + 2 * TB, wsrc + a.tile_panel + (size_t)ks * a.tile_slice, 2 * TB,
+                                 &full[st]);
                     } else {  // the two 64-row tiles of a down panel are adjacent
-                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * kTileBytes, &full[st]);
+                        bulk_g2s(W_at(st), wsrc + (size_t)ks * a.tile_slice, 2 * TB, &full[st]);
                     }
                     tma_load_2d(B_at(st), &maps.m[bsel], ks * 64, tl.y, &full[st]);
                 }
@@ -264,45 +349,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     break;
                 }
                 // row r of the 128-row block: tile half r / 64, row r % 64 of that tile
-                const uint8_t *wt = W_at(st) + (row >> 6) * (NMAT * kTileBytes) + mat * kTileBytes;
-                const int ri = row & 63;
-                const uint4 cw = *reinterpret_cast<const uint4 *>(wt + 16 * ri);
-                uint32_t scb = *reinterpret_cast<const uint32_t *>(wt + kTileScaleOffset + 4 * ri);
-                const __half2 s01 = *reinterpret_cast<__half2 *>(&scb);
-                const __half2 sh0 = __low2half2(s01), sh1 = __high2half2(s01);
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-                const uint32_t words8[4] = {cw.x >> 8, cw.y >> 8, cw.z >> 8, cw.w >> 8};
+                const uint8_t *wt = W_at(st) + (row >> 6) * (NMAT * TB) + mat * TB;
                 uint8_t *arow = A_at(st, mat) + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {  // output chunk c: columns 8c .. 8c+7
-                    if (c < c_lo || c >= c_hi) continue;
-                    const __half2 sc = (c < 4) ? sh0 : sh1;
-                    // Columns 8c + 2t, 8c + 2t + 1 (step j = c / 2, half s = c % 2)
-                    // sit in word t at bits 8s + 6 - 2j and 16 + 8s + 6 - 2j. With
-                    // the exponent that gives bit 6 - 2j the place value 1, the
-                    // masked pair reads as the exact fp16 values base_j + code
-                    // (base 16, 64, 256, 1024); subtracting base_j + 1.5 is exact
-                    // for j < 3 (17.5, 65.5, 257.5), and in two exact steps for
-                    // j = 3; one multiply by the scale rounds once.
-                    const int j = c >> 1;
-                    const uint32_t m = 0x00030003u << (6 - 2 * j);
-                    const uint32_t g = j == 0 ? 0x4C004C00u : j == 1 ? 0x54005400u : j == 2 ? 0x5C005C00u : 0x64006400u;
-                    uint32_t out[4];
-#pragma unroll
-                    for (int pr = 0; pr < 4; ++pr) {
-                        uint32_t v = (((c & 1) ? words8[pr] : words[pr]) & m) | g;
-                        __half2 h = *reinterpret_cast<__half2 *>(&v);
-                        if (j < 3) {
-                            const float off = j == 0 ? 17.5f : j == 1 ? 65.5f : 257.5f;
-                            h = __hsub2(h, __floats2half2_rn(off, off));
-                        } else {
-                            h = __hsub2(__hsub2(h, __floats2half2_rn(1024.f, 1024.f)), __floats2half2_rn(1.5f, 1.5f));
-                        }
-                        h = __hmul2(h, sc);  // (c - 1.5) s
-                        out[pr] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                    *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
-                }
+                if constexpr (BITS == 4)
+                    dequant_row_q4(wt, row & 63, c_lo, c_hi, row, arow);
+                else
+                    dequant_row_q2(wt, row & 63, c_lo, c_hi, row, arow);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&aready[st]);
@@ -318,17 +370,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
 }
 
 template <int MODE>
-static void launch_gemm(const TmaMaps &maps, const GemmArgs &a, int num_sms, cudaStream_t st) {
-    using L = GLayout<MODE>;
-    k_expert_gemm<MODE><<<num_sms, kGemmThreads, L::SMEM, st>>>(maps, a);
+static void launch_gemm(const TmaMaps &maps, const GemmArgs &a, int bits, int num_sms, cudaStream_t st) {
+    if (bits == 4)
+        k_expert_gemm<MODE, 4><<<num_sms, kGemmThreads, GLayout<MODE, 4>::SMEM, st>>>(maps, a);
+    else
+        k_expert_gemm<MODE, 2><<<num_sms, kGemmThreads, GLayout<MODE, 2>::SMEM, st>>>(maps, a);
+}
+
+template <int MODE, int BITS>
+static cudaError_t set_gemm_limit(int max_smem) {
+    if ((int)GLayout<MODE, BITS>::SMEM > max_smem) return cudaErrorInvalidValue;
+    return cudaFuncSetAttribute(k_expert_gemm<MODE, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)GLayout<MODE, BITS>::SMEM);
 }
 
 cudaError_t init_gemm_attributes(int max_smem) {
-    if ((int)GLayout<0>::SMEM > max_smem || (int)GLayout<1>::SMEM > max_smem) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)GLayout<0>::SMEM);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_expert_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GLayout<1>::SMEM);
+    cudaError_t e;
+    if ((e = set_gemm_limit<0, 2>(max_smem)) != cudaSuccess) return e;
+    if ((e = set_gemm_limit<1, 2>(max_smem)) != cudaSuccess) return e;
+    if ((e = set_gemm_limit<0, 4>(max_smem)) != cudaSuccess) return e;
+    return set_gemm_limit<1, 4>(max_smem);
 }
 
 void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps &maps, int max_tiles, int T,
@@ -350,7 +411,7 @@ void launch_expert_gemm1(const Workspace &ws, const uint8_t *blob, const TmaMaps
     a.n_pairs = T * s.k;
     a.status = ws.status;
     (void)max_tiles;
-    launch_gemm<0>(maps, a, num_sms, st);
+    launch_gemm<0>(maps, a, s.bits, num_sms, st);
 }
 
 // y[t] (+)= sum_j w_j O[pair_of(t, j)] / s_t^2: one CTA per token, 8 features
@@ -416,7 +477,7 @@ void launch_expert_gemm2(const Workspace &ws, const uint8_t *blob, float *y, con
     a.n_pairs = T * s.k;
     a.status = ws.status;
     (void)max_tiles;
-    launch_gemm<1>(maps, a, num_sms, st);
+    launch_gemm<1>(maps, a, s.bits, num_sms, st);
 }
 
 }  // namespace strata

@@ -150,7 +150,8 @@ extern "C" strata_status strata_moe_route_noalloc(const strata_moe_desc *desc, c
     if ((s = scratch_of_current_device(&base)) != STRATA_OK) return s;
     if (n_tokens == 0) return STRATA_OK;
 
-    const strata::Shape sh{desc->d_model, desc->d_ff, desc->n_experts, desc->top_k};
+    const strata::Shape sh{desc->d_model, desc->d_ff, desc->n_experts, desc->top_k,
+                           desc->weight_format == STRATA_FMT_Q4_0_TILED ? 4 : 2};
     const int P = n_tokens * sh.k;
     strata::Workspace ws{};
     ws.meta = reinterpret_cast<int32_t *>(base + kOffMeta);

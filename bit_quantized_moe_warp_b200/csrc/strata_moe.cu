@@ -60,8 +60,8 @@ extern "C" const char *strata_last_error(void) { return g_last_error; }
 
 // ------------------------------------------------------------ sizes
 namespace strata {
-size_t expert_bytes(const Shape &s) { return (size_t)3 * s.d * s.f / 32 * 10; }
-size_t down_section_offset(const Shape &s) { return (size_t)2 * s.d * s.f / 32 * 10; }
+size_t expert_bytes(const Shape &s) { return (size_t)3 * (s.d / 64) * (s.f / 64) * tile_bytes(s); }
+size_t down_section_offset(const Shape &s) { return (size_t)2 * (s.d / 64) * (s.f / 64) * tile_bytes(s); }
 }  // namespace strata
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -69,8 +69,8 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static strata_status validate_desc(const strata_moe_desc *d) {
     if (!d) return fail(STRATA_ERR_INVALID_ARG, "desc is NULL");
     if (d->block_size != 32) return fail(STRATA_ERR_UNSUPPORTED, "block_size must be 32 (got %d)", d->block_size);
-    if (d->weight_format != STRATA_FMT_Q2_0_TILED)
-        return fail(STRATA_ERR_UNSUPPORTED, "weight_format must be STRATA_FMT_Q2_0_TILED");
+    if (d->weight_format != STRATA_FMT_Q2_0_TILED && d->weight_format != STRATA_FMT_Q4_0_TILED)
+        return fail(STRATA_ERR_UNSUPPORTED, "weight_format must be STRATA_FMT_Q2_0_TILED or STRATA_FMT_Q4_0_TILED");
     if (d->d_model <= 0 || d->d_model % 128 || d->d_model > 16384)
         return fail(STRATA_ERR_INVALID_ARG, "d_model must be a positive multiple of 128 <= 16384 (got %d)",
                     d->d_model);
@@ -99,7 +99,9 @@ strata_status strata_set_error(strata_status s, const char *fmt, ...) {
 
 strata_status strata_check_desc(const strata_moe_desc *desc) { return validate_desc(desc); }
 
-static Shape shape_of(const strata_moe_desc *d) { return Shape{d->d_model, d->d_ff, d->n_experts, d->top_k}; }
+static Shape shape_of(const strata_moe_desc *d) {
+    return Shape{d->d_model, d->d_ff, d->n_experts, d->top_k, d->weight_format == STRATA_FMT_Q4_0_TILED ? 4 : 2};
+}
 
 // Workspace plan: offsets of every buffer in one allocation (256-B aligned).
 struct Plan {
@@ -290,7 +292,12 @@ extern "C" strata_status strata_moe_set_stage_events(strata_moe_layer L, void *c
 
 extern "C" size_t strata_q2_matrix_bytes(int32_t rows, int32_t K) {
     if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS) return 0;
-    return (size_t)rows * K / 64 * 20;
+    return (size_t)(rows / 64) * (K / 64) * STRATA_Q2_TILE_BYTES;
+}
+
+extern "C" size_t strata_q4_matrix_bytes(int32_t rows, int32_t K) {
+    if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS) return 0;
+    return (size_t)(rows / 64) * (K / 64) * STRATA_Q4_TILE_BYTES;
 }
 
 extern "C" size_t strata_moe_expert_bytes(const strata_moe_desc *desc) {
@@ -694,45 +701,67 @@ extern "C" strata_status strata_selftest_bounds_check(strata_stream_t stream) {
 
 // ------------------------------------------------------------ packers
 // Tile (p, s) of a [rows x K] matrix -- rows 64p.., columns 64s.. -- goes to
-// dst + p * panel_stride + s * slice_stride.
-static void pack_matrix_host(const uint8_t *codes, const uint16_t *scales, int rows, int K, uint8_t *dst,
+// dst + p * panel_stride + s * slice_stride. Column c = 16j + 8s + 2t + h of
+// a tile row: 2-bit codes in word t at bit 16h + 8s + 6 - 2j (four words);
+// 4-bit codes in word 2t + j/2 at bit 16h + 8(j%2) + 4s (eight words).
+static void pack_matrix_host(const uint8_t *codes, const uint16_t *scales, int rows, int K, int bits, uint8_t *dst,
                              size_t panel_stride, size_t slice_stride) {
+    const int nw = bits == 4 ? 8 : 4;
+    const size_t soff = bits == 4 ? Qn<4>::kScaleOffset : Qn<2>::kScaleOffset;
     for (int p = 0; p < rows / STRATA_Q2_TILE_ROWS; ++p)
         for (int s = 0; s < K / STRATA_Q2_TILE_COLS; ++s) {
             uint8_t *t = dst + (size_t)p * panel_stride + (size_t)s * slice_stride;
             for (int i = 0; i < STRATA_Q2_TILE_ROWS; ++i) {
                 const int r = p * STRATA_Q2_TILE_ROWS + i;
-                uint32_t w[4] = {0, 0, 0, 0};
-                for (int c = 0; c < 64; ++c)  // c = 16j + 8s + 2t + h -> word t, bit 16h + 8s + 6 - 2j
-                    w[(c % 8) / 2] |= (uint32_t)(codes[(size_t)r * K + 64 * s + c] & 3u)
-                                      << (16 * (c % 2) + 8 * ((c / 8) % 2) + 6 - 2 * (c / 16));
-                for (int q = 0; q < 4; ++q)
-                    for (int b = 0; b < 4; ++b) t[16 * i + 4 * q + b] = (uint8_t)(w[q] >> (8 * b));
+                uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                for (int c = 0; c < 64; ++c) {
+                    const uint32_t v = codes[(size_t)r * K + 64 * s + c];
+                    const int j = c / 16, sh = (c / 8) % 2, tq = (c % 8) / 2, h = c % 2;
+                    if (bits == 4)
+                        w[2 * tq + j / 2] |= (v & 15u) << (16 * h + 8 * (j % 2) + 4 * sh);
+                    else
+                        w[tq] |= (v & 3u) << (16 * h + 8 * sh + 6 - 2 * j);
+                }
+                for (int q = 0; q < nw; ++q)
+                    for (int b = 0; b < 4; ++b) t[4 * nw * i + 4 * q + b] = (uint8_t)(w[q] >> (8 * b));
                 for (int b = 0; b < 2; ++b) {
                     const uint16_t sv = scales[(size_t)r * (K / 32) + 2 * s + b];
-                    t[kTileScaleOffset + 4 * i + 2 * b] = (uint8_t)(sv & 0xff);
-                    t[kTileScaleOffset + 4 * i + 2 * b + 1] = (uint8_t)(sv >> 8);
+                    t[soff + 4 * i + 2 * b] = (uint8_t)(sv & 0xff);
+                    t[soff + 4 * i + 2 * b + 1] = (uint8_t)(sv >> 8);
                 }
             }
         }
 }
 
-static strata_status check_codes(const uint8_t *codes, size_t n) {
+static strata_status check_codes(const uint8_t *codes, size_t n, int bits) {
+    const unsigned top = (1u << bits) - 1u;
     for (size_t i = 0; i < n; ++i)
-        if (codes[i] > 3) return fail(STRATA_ERR_BAD_BLOB, "code %u at index %zu is not in 0..3", codes[i], i);
+        if (codes[i] > top)
+            return fail(STRATA_ERR_BAD_BLOB, "code %u at index %zu is not in 0..%u", codes[i], i, top);
+    return STRATA_OK;
+}
+
+static strata_status pack_lone_matrix(const uint8_t *codes, const uint16_t *scales, int32_t rows, int32_t K,
+                                      int bits, void *dst) {
+    if (!codes || !scales || !dst) return fail(STRATA_ERR_INVALID_ARG, "NULL pointer");
+    if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS)
+        return fail(STRATA_ERR_INVALID_ARG, "rows and K must be multiples of 64 (got %d x %d)", rows, K);
+    strata_status s = check_codes(codes, (size_t)rows * K, bits);
+    if (s != STRATA_OK) return s;
+    const size_t tb = bits == 4 ? STRATA_Q4_TILE_BYTES : STRATA_Q2_TILE_BYTES;
+    pack_matrix_host(codes, scales, rows, K, bits, static_cast<uint8_t *>(dst), (size_t)(K / STRATA_Q2_TILE_COLS) * tb,
+                     tb);
     return STRATA_OK;
 }
 
 extern "C" strata_status strata_q2_pack(const uint8_t *codes, const uint16_t *scales, int32_t rows, int32_t K,
                                         void *dst) {
-    if (!codes || !scales || !dst) return fail(STRATA_ERR_INVALID_ARG, "NULL pointer");
-    if (rows <= 0 || K <= 0 || rows % STRATA_Q2_TILE_ROWS || K % STRATA_Q2_TILE_COLS)
-        return fail(STRATA_ERR_INVALID_ARG, "rows and K must be multiples of 64 (got %d x %d)", rows, K);
-    strata_status s = check_codes(codes, (size_t)rows * K);
-    if (s != STRATA_OK) return s;
-    pack_matrix_host(codes, scales, rows, K, static_cast<uint8_t *>(dst),
-                     (size_t)(K / STRATA_Q2_TILE_COLS) * STRATA_Q2_TILE_BYTES, STRATA_Q2_TILE_BYTES);
-    return STRATA_OK;
+    return pack_lone_matrix(codes, scales, rows, K, 2, dst);
+}
+
+extern "C" strata_status strata_q4_pack(const uint8_t *codes, const uint16_t *scales, int32_t rows, int32_t K,
+                                        void *dst) {
+    return pack_lone_matrix(codes, scales, rows, K, 4, dst);
 }
 
 extern "C" strata_status strata_moe_pack_expert(const strata_moe_desc *desc, const uint8_t *gc, const uint16_t *gs,
@@ -743,14 +772,14 @@ extern "C" strata_status strata_moe_pack_expert(const strata_moe_desc *desc, con
     if (!gc || !gs || !uc || !us || !dc || !ds || !dst) return fail(STRATA_ERR_INVALID_ARG, "NULL pointer");
     const Shape sh = shape_of(desc);
     const size_t n = (size_t)sh.d * sh.f;
-    if ((s = check_codes(gc, n)) != STRATA_OK || (s = check_codes(uc, n)) != STRATA_OK ||
-        (s = check_codes(dc, n)) != STRATA_OK)
+    if ((s = check_codes(gc, n, sh.bits)) != STRATA_OK || (s = check_codes(uc, n, sh.bits)) != STRATA_OK ||
+        (s = check_codes(dc, n, sh.bits)) != STRATA_OK)
         return s;
     uint8_t *b = static_cast<uint8_t *>(dst);
     const ExpertStrides x = expert_strides(sh);
-    pack_matrix_host(gc, gs, sh.f, sh.d, b, x.gu_panel, x.gu_slice);
-    pack_matrix_host(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, x.gu_panel, x.gu_slice);
-    pack_matrix_host(dc, ds, sh.d, sh.f, b + down_section_offset(sh), x.dn_panel, x.dn_slice);
+    pack_matrix_host(gc, gs, sh.f, sh.d, sh.bits, b, x.gu_panel, x.gu_slice);
+    pack_matrix_host(uc, us, sh.f, sh.d, sh.bits, b + tile_bytes(sh), x.gu_panel, x.gu_slice);
+    pack_matrix_host(dc, ds, sh.d, sh.f, sh.bits, b + down_section_offset(sh), x.dn_panel, x.dn_slice);
     return STRATA_OK;
 }
 
@@ -766,8 +795,8 @@ extern "C" strata_status strata_moe_pack_expert_device(const strata_moe_desc *de
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *b = static_cast<uint8_t *>(dst);
     const ExpertStrides x = expert_strides(sh);
-    launch_pack_matrix_device(gc, gs, sh.f, sh.d, b, x.gu_panel, x.gu_slice, st);
-    launch_pack_matrix_device(uc, us, sh.f, sh.d, b + STRATA_Q2_TILE_BYTES, x.gu_panel, x.gu_slice, st);
-    launch_pack_matrix_device(dc, ds, sh.d, sh.f, b + down_section_offset(sh), x.dn_panel, x.dn_slice, st);
+    launch_pack_matrix_device(gc, gs, sh.f, sh.d, sh.bits, b, x.gu_panel, x.gu_slice, st);
+    launch_pack_matrix_device(uc, us, sh.f, sh.d, sh.bits, b + tile_bytes(sh), x.gu_panel, x.gu_slice, st);
+    launch_pack_matrix_device(dc, ds, sh.d, sh.f, sh.bits, b + down_section_offset(sh), x.dn_panel, x.dn_slice, st);
     return check_launch("pack kernels");
 }

@@ -92,11 +92,30 @@ typedef enum {
  * ((d/64) * 2560 bytes) and the down columns it feeds ((d/64) * 1280
  * bytes); the tensor-core path's 128-row panels are two adjacent 64-row
  * tiles (down) or two 2560-byte pairs (gate/up).
+ *
+ * STRATA_FMT_Q4_0_TILED: the 4-bit block level. The pages' quality ladder
+ * (first page, 能跑多快, its table: Q2_0, IQ2_XS, IQ3_XXS, IQ3_S) has wider
+ * levels but does not print their bits; this one is the 2-bit rule with
+ * 4-bit codes, this library's own:
+ *   weight W[r][k] = (c[r][k] - 7.5) * s[r][k/32], c in {0..15}, s fp16.
+ * The same 64 x 64 tiles, 2304 bytes each:
+ *   bytes [0, 2048):   codes, row i at bytes 32i..32i+31, eight
+ *                      little-endian uint32 words W0..W7; column
+ *                      c = 16j + 8s + 2t + h lives in word W(2t + j/2) at
+ *                      bits 16h + 8(j%2) + 4s .. +3. Lane t of a 4-lane
+ *                      group reads W(2t), W(2t+1) (one 8-byte load) and
+ *                      holds every code of its fragment columns; one mask
+ *                      per register extracts a column pair;
+ *   bytes [2048, 2304): scales, row i at 2048+4i, as in the 2-bit tile.
+ * Expert blob and tile order as above with 2304-byte tiles: gate/up pairs of
+ * 4608 bytes, 3*d*f/32*18 bytes per expert (d=2048, f=768: 2,654,208).
  */
 #define STRATA_FMT_Q2_0_TILED 1
+#define STRATA_FMT_Q4_0_TILED 2
 #define STRATA_Q2_TILE_ROWS 64
 #define STRATA_Q2_TILE_COLS 64
 #define STRATA_Q2_TILE_BYTES 1280
+#define STRATA_Q4_TILE_BYTES 2304
 
 /* desc.flags */
 #define STRATA_ACCUMULATE 1u      /* y += MoE(x) instead of y = MoE(x) */
@@ -112,16 +131,18 @@ typedef struct {
     int32_t top_k;        /* k, 1 <= k <= min(E, 32) */
     int32_t max_tokens;   /* largest n_tokens of one layer call (workspace size) */
     int32_t block_size;   /* must be 32 */
-    int32_t weight_format;/* must be STRATA_FMT_Q2_0_TILED */
+    int32_t weight_format;/* STRATA_FMT_Q2_0_TILED or STRATA_FMT_Q4_0_TILED */
     uint32_t flags;       /* STRATA_ACCUMULATE | STRATA_FORCE_PREFILL */
     const float *router_bias; /* device fp32 [E] added to the logits, or NULL */
 } strata_moe_desc;
 
 typedef struct strata_moe_layer_s *strata_moe_layer;
 
-/* Bytes of one packed matrix [rows x K] (rows % 64 == 0, K % 64 == 0). */
+/* Bytes of one packed matrix [rows x K] (rows % 64 == 0, K % 64 == 0), 2-bit
+ * and 4-bit format; 0 for other shapes. */
 size_t strata_q2_matrix_bytes(int32_t rows, int32_t K);
-/* Bytes of one packed expert: 3*d*f/32*10. */
+size_t strata_q4_matrix_bytes(int32_t rows, int32_t K);
+/* Bytes of one packed expert: 3*d*f/32*10 (2-bit), 3*d*f/32*18 (4-bit). */
 size_t strata_moe_expert_bytes(const strata_moe_desc *desc);
 /* Bytes of the whole expert blob of a layer: E * strata_moe_expert_bytes. */
 size_t strata_moe_expert_blob_bytes(const strata_moe_desc *desc);
@@ -257,16 +278,22 @@ strata_status strata_moe_check_status(strata_moe_layer layer);
  * Errors: BAD_BLOB (a code > 3), INVALID_ARG. */
 strata_status strata_q2_pack(const uint8_t *codes, const uint16_t *scales_fp16, int32_t rows,
                              int32_t K, void *dst);
+/* The same for the 4-bit format: codes 0..15, dst strata_q4_matrix_bytes.
+ * Errors: BAD_BLOB (a code > 15), INVALID_ARG. */
+strata_status strata_q4_pack(const uint8_t *codes, const uint16_t *scales_fp16, int32_t rows,
+                             int32_t K, void *dst);
 
 /* Pack one expert on the HOST into its blob section (dst: host,
- * strata_moe_expert_bytes): gate/up [f x d], down [d x f]. */
+ * strata_moe_expert_bytes) in desc->weight_format: gate/up [f x d], down
+ * [d x f], one code per byte (0..3 or 0..15). Errors: BAD_BLOB (a code out
+ * of range), INVALID_ARG, UNSUPPORTED (desc). */
 strata_status strata_moe_pack_expert(const strata_moe_desc *desc, const uint8_t *gate_codes,
                                      const uint16_t *gate_scales, const uint8_t *up_codes,
                                      const uint16_t *up_scales, const uint8_t *down_codes,
                                      const uint16_t *down_scales, void *dst);
 
 /* Same as strata_moe_pack_expert with device pointers, on `stream`. Codes
- * above 3 are masked to 2 bits. */
+ * above the format's largest (3 or 15) are masked to its 2 or 4 bits. */
 strata_status strata_moe_pack_expert_device(const strata_moe_desc *desc, const uint8_t *gate_codes,
                                             const uint16_t *gate_scales, const uint8_t *up_codes,
                                             const uint16_t *up_scales, const uint8_t *down_codes,

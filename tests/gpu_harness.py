@@ -29,12 +29,14 @@ def S():
 class HostLayer:
     """All inputs of one layer generated on the host (small shapes)."""
 
-    def __init__(self, d, f, E, k, T, seed=0, layer=0, zipf=False, experts=None, W=None, x=None, bias=None):
-        self.d, self.f, self.E, self.k, self.T = d, f, E, k, T
+    def __init__(self, d, f, E, k, T, seed=0, layer=0, zipf=False, experts=None, W=None, x=None, bias=None,
+                 bits=2):
+        self.d, self.f, self.E, self.k, self.T, self.bits = d, f, E, k, T, bits
         self.x = synth.gen_x_bf16(seed, T, d) if x is None else x
         self.W = synth.gen_router_w(seed, layer, E, d) if W is None else W
         self.bias = (synth.gen_zipf_bias(seed, layer, E) if zipf else None) if bias is None else bias
-        self.experts = [synth.gen_expert(seed, layer, e, d, f) for e in range(E)] if experts is None else experts
+        self.experts = ([synth.gen_expert(seed, layer, e, d, f, bits) for e in range(E)]
+                        if experts is None else experts)
 
     def blob(self, desc):
         eb = S().strata_moe_expert_bytes(desc)
@@ -72,7 +74,7 @@ def expert_source(w: synth.Workload, layer: int):
 
     def get(e):
         if e not in cache:
-            cache[e] = synth.gen_expert(w.seed, layer, e, w.d, w.f)
+            cache[e] = synth.gen_expert(w.seed, layer, e, w.d, w.f, w.bits)
         return cache[e]
 
     return get

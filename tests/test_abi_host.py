@@ -50,6 +50,28 @@ def test_pack_golden_tile(S):
     assert np.array_equal(out, blob), "library packer differs from the hand-worked tile"
 
 
+def test_pack_golden_q4_tile(S):
+    blob, expects = pins_lib.load_tile_example("q4_tile_example.txt", 2304)
+    codes, scales = oracle.unpack_q4_tiled(blob, 64, 64)
+    out = np.zeros(2304, np.uint8)
+    S.strata_q4_pack(codes, scales, 64, 64, out)
+    assert np.array_equal(out, blob), "library packer differs from the hand-worked 4-bit tile"
+
+
+@pytest.mark.parametrize("rows,K", [(64, 64), (128, 64), (256, 128), (64, 768), (384, 256)])
+def test_pack_roundtrip_q4_matrix(S, rows, K):
+    rng = np.random.default_rng(rows * 11 + K)
+    codes = rng.integers(0, 16, (rows, K), dtype=np.uint8)
+    scales = (rng.standard_normal((rows, K // 32)) * 0.02).astype(np.float16)
+    n = S.strata_q4_matrix_bytes(rows, K)
+    assert n == rows * K // 64 * 36
+    out = np.zeros(n, np.uint8)
+    S.strata_q4_pack(codes, scales, rows, K, out)
+    c2, s2 = oracle.unpack_q4_tiled(out, rows, K)
+    assert np.array_equal(c2, codes)
+    assert np.array_equal(s2.view(np.uint16), scales.view(np.uint16))
+
+
 @pytest.mark.parametrize("rows,K", [(64, 64), (128, 64), (256, 128), (64, 768), (384, 256)])
 def test_pack_roundtrip_matrix(S, rows, K):
     rng = np.random.default_rng(rows * 7 + K)
@@ -64,17 +86,18 @@ def test_pack_roundtrip_matrix(S, rows, K):
     assert np.array_equal(s2.view(np.uint16), scales.view(np.uint16))
 
 
-def test_pack_expert_layout(S):
+@pytest.mark.parametrize("bits", [2, 4])
+def test_pack_expert_layout(S, bits):
     d, f = 256, 128
-    desc = S.make_desc(d, f, 4, 2, 8)
-    ex = synth.gen_expert(5, 0, 3, d, f)
+    desc = S.make_desc(d, f, 4, 2, 8, bits=bits)
+    ex = synth.gen_expert(5, 0, 3, d, f, bits)
     eb = S.strata_moe_expert_bytes(desc)
-    assert eb == 3 * d * f // 32 * 10
+    assert eb == 3 * d * f // 32 * (10 if bits == 2 else 18)
     out = np.zeros(eb, np.uint8)
     S.strata_moe_pack_expert(desc, ex["gate_codes"], ex["gate_scales"], ex["up_codes"], ex["up_scales"],
                              ex["down_codes"], ex["down_scales"], out)
-    got = oracle.unpack_expert(out, d, f)
-    assert got["bits"] == ex["bits"] == 2
+    got = oracle.unpack_expert(out, d, f, bits)
+    assert got["bits"] == ex["bits"] == bits
     for key in ex:
         if key == "bits":
             continue
@@ -89,6 +112,18 @@ def test_pack_rejects_bad_code(S):
     codes[3, 5] = 4
     with pytest.raises(S.StrataError) as ei:
         S.strata_q2_pack(codes, np.zeros((128, 2), np.float16), 128, 64, np.zeros(2560, np.uint8))
+    assert ei.value.status == S.STRATA_ERR_BAD_BLOB
+    S.strata_q4_pack(codes, np.zeros((128, 2), np.float16), 128, 64, np.zeros(4608, np.uint8))  # 4 is a 4-bit code
+    codes[3, 5] = 16
+    with pytest.raises(S.StrataError) as ei:
+        S.strata_q4_pack(codes, np.zeros((128, 2), np.float16), 128, 64, np.zeros(4608, np.uint8))
+    assert ei.value.status == S.STRATA_ERR_BAD_BLOB
+    d, f = 128, 128
+    desc = S.make_desc(d, f, 4, 2, 8, bits=2)
+    big = np.full((f, d), 7, np.uint8)
+    sc = np.zeros((f, d // 32), np.float16)
+    with pytest.raises(S.StrataError) as ei:
+        S.strata_moe_pack_expert(desc, big, sc, big, sc, big.T.copy(), sc, np.zeros(3 * d * f // 32 * 10, np.uint8))
     assert ei.value.status == S.STRATA_ERR_BAD_BLOB
 
 
@@ -107,7 +142,14 @@ def test_desc_validation(S):
     d2 = S.make_desc(256, 128, 16, 4, 8)
     d2.block_size = 16
     assert S.strata_moe_workspace_bytes(d2) == 0
+    d3 = S.make_desc(256, 128, 16, 4, 8)
+    d3.weight_format = 3
+    assert S.strata_moe_workspace_bytes(d3) == 0
     assert S.strata_q2_matrix_bytes(100, 64) == 0
+    assert S.strata_q4_matrix_bytes(64, 100) == 0
+    q4 = S.make_desc(2048, 768, 512, 10, 8192, bits=4)
+    assert S.strata_moe_expert_bytes(q4) == 2654208
+    assert S.strata_moe_workspace_bytes(q4) == S.strata_moe_workspace_bytes(ok)
 
 
 def test_status_strings(S):
@@ -121,7 +163,8 @@ def test_binding_constants_match_header(S):
     defs = dict(re.findall(r"#define\s+(STRATA_[A-Z0-9_]+)\s+\(?([0-9]+)u?\b", src))
     restated = [n for n in dir(S) if n.startswith("STRATA_") and n in defs]
     assert {"STRATA_Q2_TILE_BYTES", "STRATA_ACCUMULATE", "STRATA_FORCE_PREFILL",
-            "STRATA_DECODE_MAX_TOKENS", "STRATA_FMT_Q2_0_TILED"} <= set(restated)
+            "STRATA_DECODE_MAX_TOKENS", "STRATA_FMT_Q2_0_TILED", "STRATA_FMT_Q4_0_TILED",
+            "STRATA_Q4_TILE_BYTES"} <= set(restated)
     for n in restated:
         assert getattr(S, n) == int(defs[n]), n
 

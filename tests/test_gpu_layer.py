@@ -20,7 +20,7 @@ def run_layer(h: HostLayer, flags=0, max_tokens=None, y0=None):
     mt = max_tokens or max(h.T, 1)
     dev = torch_dev()
     bias_d = None if h.bias is None else torch.from_numpy(h.bias).to(dev)
-    layer = lib.MoELayer(h.d, h.f, h.E, h.k, mt, flags=flags, router_bias=bias_d)
+    layer = lib.MoELayer(h.d, h.f, h.E, h.k, mt, flags=flags, router_bias=bias_d, bits=h.bits)
     xd, Wd, _, blob = h.to_device(layer.desc)
     y = torch.zeros((h.T, h.d), dtype=torch.float32, device=dev) if y0 is None else torch.from_numpy(y0).to(dev)
     layer.forward(xd, Wd, blob, y, h.T)
@@ -234,7 +234,7 @@ def full_size_check(w: synth.Workload, T: int, flags: int, sample: int, layer_id
     W = synth.gen_router_w(w.seed, layer_idx, w.E, w.d)
     bias = synth.router_bias(w, layer_idx)
     bias_d = None if bias is None else torch.from_numpy(bias).to(dev)
-    layer = lib.MoELayer(w.d, w.f, w.E, w.k, T, flags=flags, router_bias=bias_d)
+    layer = lib.MoELayer(w.d, w.f, w.E, w.k, T, flags=flags, router_bias=bias_d, bits=w.bits)
     blob = device_blob(w, layer_idx, layer.desc)
     xd = torch.from_numpy(x.view(np.int16)).to(dev)
     Wd = torch.from_numpy(W).to(dev)
@@ -294,3 +294,50 @@ def test_prefill_layer_8192_sampled():
     expert outputs on 48 sampled tokens."""
     e, nex = full_size_check(synth.WORKLOADS["prefill"], 8192, 0, 48)
     print(f"prefill T=8192: max row err {e:.2e}, exempt {nex}")
+
+
+# ---------------------------------------------------------------- 4-bit format
+
+
+@pytest.mark.parametrize("flags", [0, 2], ids=["decode", "prefill"])
+def test_tiny_layer_q4(flags):
+    h = HostLayer(256, 128, 16, 4, 8, seed=4, bits=4)
+    err = check_full(h, run_layer(h, flags))
+    print(f"tiny 4-bit flags={flags}: max row err {err.max():.2e}")
+
+
+Q4_SHAPES = [
+    # d, f, E, k, T, zipf, flags
+    (256, 128, 16, 4, 1, False, 0),
+    (384, 256, 64, 10, 16, True, 0),
+    (256, 256, 64, 10, 17, True, 0),   # first prefill size
+    (512, 128, 64, 4, 130, True, 0),   # ragged tiles
+    (128, 256, 16, 2, 1000, True, 0),  # several 128/256-token tiles per expert
+    (256, 128, 16, 4, 5, False, 2),    # tensor-core path at a decode size
+]
+
+
+@pytest.mark.parametrize("d,f,E,k,T,zipf,flags", Q4_SHAPES)
+def test_shapes_q4(d, f, E, k, T, zipf, flags):
+    h = HostLayer(d, f, E, k, T, seed=3 * d + f + E + k + T, zipf=zipf, bits=4)
+    err = check_full(h, run_layer(h, flags), exact_routing=False)
+    print(f"4-bit {d}x{f} E={E} k={k} T={T}: max row err {err.max():.2e}")
+
+
+def test_decode_layer_full_size_q4():
+    """4-bit experts: one token, 512 experts, top-10 (d=2048, f=768)."""
+    e, nex = full_size_check(synth.WORKLOADS["decode_q4"], 1, 0, 1)
+    print(f"4-bit decode T=1: max row err {e:.2e}")
+
+
+@pytest.mark.parametrize("T", [4, 16])
+def test_verify_layer_full_size_q4(T):
+    e, nex = full_size_check(synth.WORKLOADS["verify4_q4"], T, 0, T)
+    print(f"4-bit verify T={T}: max row err {e:.2e}, exempt {nex}")
+
+
+def test_prefill_layer_8192_sampled_q4():
+    """4-bit experts, 8,192-token chunk with Zipf routing: every token's
+    routing, expert outputs on 48 sampled tokens."""
+    e, nex = full_size_check(synth.WORKLOADS["prefill_q4"], 8192, 0, 48)
+    print(f"4-bit prefill T=8192: max row err {e:.2e}, exempt {nex}")

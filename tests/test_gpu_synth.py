@@ -17,20 +17,22 @@ def test_device_generator_matches_host():
     assert np.array_equal(x, synth.gen_x_bf16(3, 5, 256, tok0=7))
     W = sd.router_w(2, 4, 64, 128).cpu().numpy()
     assert np.array_equal(W, synth.gen_router_w(2, 4, 64, 128))
-    for mat, rows, K in ((synth.GATE, 768, 2048), (synth.DOWN, 256, 128)):
-        c, s = sd.expert_codes_scales(1, 3, [0, 17, 511], mat, rows, K)
-        c, s = c.cpu().numpy(), s.cpu().numpy().view(np.uint16)
-        for i, e in enumerate([0, 17, 511]):
-            assert np.array_equal(c[i], synth.gen_codes(1, 3, e, mat, rows, K))
-            assert np.array_equal(s[i], synth.gen_scales(1, 3, e, mat, rows, K).view(np.uint16))
+    for bits in (2, 4):
+        for mat, rows, K in ((synth.GATE, 768, 2048), (synth.DOWN, 256, 128)):
+            c, s = sd.expert_codes_scales(1, 3, [0, 17, 511], mat, rows, K, bits)
+            c, s = c.cpu().numpy(), s.cpu().numpy().view(np.uint16)
+            for i, e in enumerate([0, 17, 511]):
+                assert np.array_equal(c[i], synth.gen_codes(1, 3, e, mat, rows, K, bits))
+                assert np.array_equal(s[i], synth.gen_scales(1, 3, e, mat, rows, K, bits).view(np.uint16))
 
 
-def test_device_packer_matches_host_packer():
+@pytest.mark.parametrize("bits", [2, 4])
+def test_device_packer_matches_host_packer(bits):
     import torch
     lib = S()
     d, f = 512, 256
-    desc = lib.make_desc(d, f, 4, 2, 8)
-    ex = synth.gen_expert(9, 0, 1, d, f)
+    desc = lib.make_desc(d, f, 4, 2, 8, bits=bits)
+    ex = synth.gen_expert(9, 0, 1, d, f, bits)
     eb = lib.strata_moe_expert_bytes(desc)
     host = np.zeros(eb, np.uint8)
     lib.strata_moe_pack_expert(desc, ex["gate_codes"], ex["gate_scales"], ex["up_codes"], ex["up_scales"],
@@ -42,7 +44,7 @@ def test_device_packer_matches_host_packer():
                                       t(ex["up_scales"]), t(ex["down_codes"]), t(ex["down_scales"]), out)
     torch.cuda.synchronize()
     assert np.array_equal(out.cpu().numpy(), host)
-    got = oracle.unpack_expert(host, d, f)
+    got = oracle.unpack_expert(host, d, f, bits)
     assert np.array_equal(got["down_codes"], ex["down_codes"])
 
 
