@@ -143,6 +143,13 @@ STRATA_DEV void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Programmatic dependent launch: wait until the grids this launch depends on
+// have completed and their memory is visible (a no-op for a launch without
+// the programmatic-serialization attribute), and let the launches that depend
+// on this grid start once every CTA has signalled or exited.
+STRATA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+STRATA_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // generic-proxy smem writes -> visible to the async proxy (tensor core, TMA)
 STRATA_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -13,14 +13,17 @@
 //            zero the CTA's slice of y, stage x as fp16 (or bf16(RMSNorm) of
 //            the fp32 residual, the stack glue), compute the router partial
 //            sums of their rows in K quarters and reduce them, in a fixed
-//            order, plus the bias, into the logits; grid barrier.
+//            order, plus the bias, into the logits; grid barrier, during
+//            which the other warps compute the per-block constants of x.
 //   phase 1  every CTA reads all logits and computes, redundantly and
-//            identically, each token's softmax top-k (one warp per token,
-//            per-lane sorted lists, one warp max and a ballot per pick, ties
-//            to the lower expert index), the renormalised weights and the
-//            per-expert token lists (bit masks of tokens, popcount ranks);
-//            warps without a token meanwhile compute the per-block constants
-//            of x. CTA 0 publishes the routing.
+//            identically, each token's softmax top-k (logit descending, ties
+//            to the lower expert index). The k-th largest of 16 group maxima
+//            bounds the token's k-th largest logit from below; the logits at
+//            or above it are the candidates, and each candidate's rank is the
+//            number of candidates that beat it. Then the renormalised weights
+//            and the per-expert token lists (bit masks of tokens, scans over
+//            the experts, popcount ranks). The CTA with the least expert work
+//            publishes the routing at its end.
 //   phase 2  work units (active expert e, 64-row slice p of its hidden
 //            layer), dealt round-robin over the CTAs. A unit needs no other
 //            unit: it streams the slice's gate and up rows over all of K
@@ -109,8 +112,13 @@ __host__ __device__ inline int hstride(int n) { return n + 8; }
 
 // shared-memory plan, identical on host and device
 struct FusedSmem {
-    size_t xh, xz, red, hh, hz, lsm, sbias, sel_idx, sel_val, sel_w, mask, cnt, off, act, ptok, pslot, pw, scan, bufs, total;
+    size_t xh, xz, red, hh, hz, lsm, sbias, sel_idx, sel_val, sel_w, gmax, ccnt, mask, prank, cnt, off, act, ptok, pslot,
+        pw, scan, bufs, total;
 };
+
+// routing candidates kept per token (the selection falls back to an exact
+// one-warp pass for a token with more)
+constexpr int kCandMax = 64;
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~(size_t)15; }
 
@@ -134,7 +142,10 @@ __host__ __device__ inline FusedSmem fused_plan(int T, int TT, int d, int E, int
     p.sel_idx = o; o = al16(o + (size_t)T * k * 4);
     p.sel_val = o; o = al16(o + (size_t)T * k * 4);
     p.sel_w = o;   o = al16(o + (size_t)T * k * 4);
-    p.mask = o;    o = al16(o + (size_t)E * 4);
+    p.gmax = o;    o = al16(o + (size_t)kDecMaxT * 16 * 4);   // 16 group maxima per token (selection)
+    p.ccnt = o;    o = al16(o + (size_t)kDecMaxT * 4);        // candidates per token
+    p.mask = o;    o = al16(o + (size_t)E * 4);               // tokens of each expert (bit mask)
+    p.prank = o;   o = al16(o + (size_t)T * k * 4);           // sorted position of each pair
     p.cnt = o;     o = al16(o + (size_t)E * 4);
     p.off = o;     o = al16(o + (size_t)(E + 1) * 4);
     p.act = o;     o = al16(o + (size_t)E * 4);
@@ -394,12 +405,19 @@ STRATA_DEV void down_rows(const TileRows<BITS> &w, const uint32_t (&bf)[NT][4][2
         reinterpret_cast<float(&)[NTA][4]>(o));
 }
 
+// The exact one-warp selection, kept out of line: it runs only for k > 16 or
+// a token with more than kCandMax candidates, and inline its unrolled code
+// would sit between the selection's common steps.
+__device__ __noinline__ void token_topk_exact(const float *logits, int t, int E, int k, int *sel_idx, float *sel_val) {
+    token_topk<16>(logits, t, E, k, sel_idx, sel_val);
+}
+
 template <int TT, int BITS>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedArgs a) {
     using CC = ChunkCfg<BITS>;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar;
-    __shared__ int s_abort;
+    __shared__ int s_abort, s_nact;
     // per token: the power-of-two scale s of its staged x and 1 / s (exact);
     // per sorted pair: the routing weight / s^2 of its token
     __shared__ float xsc[kDecMaxT], xin[kDecMaxT], pws[kDecMaxT * 32];
@@ -420,14 +438,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     int *sel_idx = reinterpret_cast<int *>(smem + sp.sel_idx);
     float *sel_val = reinterpret_cast<float *>(smem + sp.sel_val);
     float *sel_w = reinterpret_cast<float *>(smem + sp.sel_w);
+    uint32_t *gmax = reinterpret_cast<uint32_t *>(smem + sp.gmax);
+    int *ccnt = reinterpret_cast<int *>(smem + sp.ccnt);
     uint32_t *mask = reinterpret_cast<uint32_t *>(smem + sp.mask);
+    int *prank = reinterpret_cast<int *>(smem + sp.prank);
+    int *scan = reinterpret_cast<int *>(smem + sp.scan);
     int *cnt = reinterpret_cast<int *>(smem + sp.cnt);
     int *off = reinterpret_cast<int *>(smem + sp.off);
     int *act = reinterpret_cast<int *>(smem + sp.act);
     int *ptok = reinterpret_cast<int *>(smem + sp.ptok);
     int *pslot = reinterpret_cast<int *>(smem + sp.pslot);
     float *pw = reinterpret_cast<float *>(smem + sp.pw);
-    int *scan = reinterpret_cast<int *>(smem + sp.scan);
     uint8_t *bufs = smem + sp.bufs;
     float *logits = a.ws.lpart;  // router logits [T][E] (+ bias)
     float *lsm = reinterpret_cast<float *>(smem + sp.lsm);
@@ -445,6 +466,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     const bool xstaged = !a.rms && xbytes <= ring;
     const uint32_t woff = xstaged ? xoff : 0u;
     const bool wstaged = nr > 0 && woff + wbytes <= ring;
+    // Launched as a dependent of the previous kernel on the stream, this CTA
+    // may start while that kernel still runs: only prefetch the router rows
+    // into L2 (a hint, harmless whoever writes them), then wait for it to
+    // finish before reading or writing anything else.
+    if (tid == 0 && nr > 0) prefetch_l2(a.W + (size_t)r0 * d, wbytes);
+    griddep_wait();
+    griddep_launch_dependents();
     if (warp == kFusedComputeWarps && lane == 0) {
         for (int i = 0; i < a.nbuf; ++i) {
             mbar_init(&full[i], 1);
@@ -453,6 +481,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         mbar_init(&xbar, 1);
         mbar_init(&wbar, 1);
         s_abort = 0;
+        s_nact = 0;
         fence_mbar_init();
         if (xstaged) {
             mbar_arrive_expect_tx(&xbar, xbytes);
@@ -603,32 +632,100 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     }
     __syncthreads();
     if (tid == 0) {  // grid barrier (release our partial logits, acquire everyone's)
-        __threadfence();
-        atomicAdd(&sync[0], 1u);
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&sync[0]) : "memory");
         wait_counter(&sync[0], (uint32_t)G, status, &s_abort);
+    } else if (!producer && warp > 0) {
+        // meanwhile the per-block constants of x (used in phase 2), in pieces
+        // of 256 columns of one token over warps 1..15
+        const int pieces = (d + 255) / 256;
+        for (int u = warp - 1; u < T * pieces; u += kFusedComputeWarps - 1) {
+            const int r = u / pieces, c0 = (u % pieces) * 256;
+            row_block_constants<BITS>(xh + (size_t)r * dpx + c0, min(256, d - c0), xz + (size_t)r * (d / 32) + c0 / 32);
+        }
     }
     __syncthreads();
 
     // ---------------------------------------------------------------- phase 1
+    constexpr int GW = kFusedComputeWarps / TT;  // warps per token in the selection; each takes TT groups
     if (!s_abort && !producer) {
         for (int e = tid; e < E; e += 512) mask[e] = 0u;
-        if (warp < T) {  // one warp per token
-            token_topk<16>(logits, warp, E, k, sel_idx + warp * k, sel_val + warp * k);
-            __syncwarp();
-            // renormalised softmax weights over the k selected
-            const float vmax = sel_val[warp * k];
-            float ex = 0.f;
-            for (int j = lane; j < k; j += 32) ex += expf(sel_val[warp * k + j] - vmax);
-            const float den = warp_sum(ex);
-            for (int j = lane; j < k; j += 32) sel_w[warp * k + j] = expf(sel_val[warp * k + j] - vmax) / den;
-        } else {  // warps without a token meanwhile compute the per-block constants of x (used in phase 2)
-            for (int r = warp - T; r < T; r += kFusedComputeWarps - T)
-                row_block_constants<BITS>(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
+        if (tid < kDecMaxT) ccnt[tid] = 0;
+        const bool fast = k <= 16;  // the bound needs k group maxima
+        const int t = warp / GW, g = warp % GW;
+        // Selection, step 1: group q of token t is experts [qE/16, (q+1)E/16)
+        // (at most 32); warp (t, g) takes groups g TT .. g TT + TT - 1, one
+        // logit of each per lane, and writes their maxima.
+        uint32_t key[TT];
+        if (fast && t < T) {
+            const float *row = logits + (size_t)t * E;
+#pragma unroll
+            for (int r = 0; r < TT; ++r) {
+                const int q = g * TT + r, lo = q * E / 16, hi = (q + 1) * E / 16;
+                key[r] = lo + lane < hi ? ordered_key(__ldcg(row + lo + lane)) : 0u;  // 0: below every real key
+            }
+#pragma unroll
+            for (int r = 0; r < TT; ++r) {
+                const uint32_t m = __reduce_max_sync(0xffffffffu, key[r]);
+                if (lane == 0) gmax[t * 16 + g * TT + r] = m;
+            }
         }
-        if (T >= kFusedComputeWarps)  // no warp was free
-            for (int r = warp; r < T; r += kFusedComputeWarps)
-                row_block_constants<BITS>(xh + (size_t)r * dpx, d, xz + (size_t)r * (d / 32));
         compute_sync();
+        // Step 2: tau = the k-th largest group maximum; the k maxima at or
+        // above it are k distinct logits, so the k-th largest logit is >= tau
+        // and every logit >= tau is a candidate (at most kCandMax kept).
+        uint2 *cand = reinterpret_cast<uint2 *>(bufs);  // [token][kCandMax] (key, expert); the ring is idle here
+        if (fast && t < T) {
+            const uint32_t mine = lane < 16 ? gmax[t * 16 + lane] : 0u;
+            int rank = 0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const uint32_t o = gmax[t * 16 + q];
+                rank += (o > mine) || (o == mine && q < lane);
+            }
+            const uint32_t hit = __ballot_sync(0xffffffffu, lane < 16 && rank == k - 1);
+            const uint32_t tau = __shfl_sync(0xffffffffu, mine, __ffs(hit) - 1);
+#pragma unroll
+            for (int r = 0; r < TT; ++r) {
+                const int lo = (g * TT + r) * E / 16;
+                const bool c = key[r] != 0u && key[r] >= tau;
+                const uint32_t bal = __ballot_sync(0xffffffffu, c);
+                if (bal) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&ccnt[t], __popc(bal));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const int pos = base + __popc(bal & ((1u << lane) - 1u));
+                    if (c && pos < kCandMax) cand[t * kCandMax + pos] = make_uint2(key[r], (uint32_t)(lo + lane));
+                }
+            }
+        }
+        compute_sync();
+        // Step 3: a candidate's place is the number of candidates that beat it
+        // (larger key, or equal key and lower expert).
+        for (int i = tid; i < T * kCandMax; i += 512) {
+            const int tt = i / kCandMax, c = i % kCandMax, C = ccnt[tt];
+            if (!fast || C > kCandMax || c >= C) continue;
+            const uint2 *cl = cand + tt * kCandMax;
+            const uint2 me = cl[c];
+            int rank = 0;
+#pragma unroll 8
+            for (int q = 0; q < C; ++q) {
+                const uint2 o = cl[q];
+                rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+            }
+            if (rank < k) {
+                sel_idx[tt * k + rank] = (int)me.y;
+                sel_val[tt * k + rank] = key_value(me.x);
+            }
+        }
+        if (warp < T && (!fast || ccnt[warp] > kCandMax))  // exact one-warp selection instead
+            token_topk_exact(logits, warp, E, k, sel_idx + warp * k, sel_val + warp * k);
+        compute_sync();
+        if (warp < T) {  // renormalised softmax weights over the token's k selected (k <= 32)
+            const float vmax = sel_val[warp * k];
+            const float ex = lane < k ? expf(sel_val[warp * k + lane] - vmax) : 0.f;
+            const float den = warp_sum(ex);
+            if (lane < k) sel_w[warp * k + lane] = ex / den;
+        }
         for (int i = tid; i < T * k; i += 512)
             if (in_bounds(sel_idx[i], E, status)) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
         compute_sync();
@@ -679,39 +776,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 off[e0 + 1] = ic + c0;
                 if (a1) act[ia + a0] = e0 + 1;
             }
-            if (tid == 0) off[E] = scan[kFusedComputeWarps - 1];
+            if (tid == 0) {
+                off[E] = scan[kFusedComputeWarps - 1];
+                s_nact = scan[32 + kFusedComputeWarps - 1];
+            }
         }
         compute_sync();
         for (int p = tid; p < T * k; p += 512) {  // pairs in (expert, ascending token) order
-            const int t = p / k, j = p % k, e = sel_idx[p];
+            const int t = p / k, e = sel_idx[p];
+            prank[p] = -1;
             if (!in_bounds(e, E, status)) continue;
             const int pos = off[e] + __popc(mask[e] & ((1u << t) - 1u));
             if (!in_bounds(pos, T * k, status)) continue;
+            prank[p] = pos;
             ptok[pos] = t;
-            pslot[pos] = j;
+            pslot[pos] = p % k;
             pw[pos] = sel_w[p];
             pws[pos] = sel_w[p] * xin[t] * xin[t];  // the down products carry s^2 of the token
-            if (b == 0) a.ws.pair_of[p] = pos;
-        }
-        compute_sync();
-        if (b == 0) {  // publish the routing of this call
-            for (int i = tid; i < T * k; i += 512) {
-                a.ws.topk_idx[i] = sel_idx[i];
-                a.ws.topk_w[i] = sel_w[i];
-                a.ws.token_list[i] = ptok[i];
-                a.ws.pair_slot[i] = pslot[i];
-                a.ws.pair_w[i] = pw[i];
-            }
-            for (int e = tid; e <= E; e += 512) a.ws.offsets[e] = off[e];
-            for (int e = tid; e < E; e += 512) a.ws.counts[e] = cnt[e];
-            if (tid == 0) {
-                a.ws.meta[META_N_ACTIVE] = scan[32 + kFusedComputeWarps - 1];
-                a.ws.meta[META_N_TOKENS] = T;
-            }
         }
     }
     __syncthreads();
-    const int n_act = s_abort ? 0 : scan[32 + kFusedComputeWarps - 1];
+    const int n_act = s_abort ? 0 : s_nact;
 
     // ---------------------------------------------------------------- phase 2
     const int FP = f / 64;   // 64-row slices of the hidden layer
@@ -946,6 +1031,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         // (stop), or none did and all of them meet here once.
         if (!stop) compute_sync_any(bad);
     }
+    __syncthreads();
+    if (b == G - 1 && !s_abort) {
+        // The routing of this call, published by the CTA dealt the fewest units.
+        for (int e = tid; e <= E; e += kFusedThreads) a.ws.offsets[e] = off[e];
+        for (int e = tid; e < E; e += kFusedThreads) a.ws.counts[e] = cnt[e];
+        if (tid == 0) {
+            a.ws.meta[META_N_ACTIVE] = n_act;
+            a.ws.meta[META_N_TOKENS] = T;
+        }
+        for (int i = tid; i < T * k; i += kFusedThreads) {
+            a.ws.topk_idx[i] = sel_idx[i];
+            a.ws.topk_w[i] = sel_w[i];
+            a.ws.token_list[i] = ptok[i];
+            a.ws.pair_slot[i] = pslot[i];
+            a.ws.pair_w[i] = pw[i];
+            a.ws.pair_of[i] = prank[i];
+        }
+    }
     // the last CTA out clears the counters for the next launch
     __syncthreads();
     if (tid == 0) {
@@ -1067,11 +1170,15 @@ cudaError_t launch_decode_fused(const Workspace &ws, const void *x, const float 
     cfg.blockDim = dim3(kFusedThreads);
     cfg.dynamicSmemBytes = c.smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    // programmatic dependent launch: this grid is set up while the previous
+    // kernel on the stream finishes (the kernel waits for it before its work)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const int slot = slot_of(T, s.bits);
     cudaError_t e = ensure_limit(slot, (int)c.smem);  // a no-op after layer creation
     if (e != cudaSuccess) return e;

@@ -269,6 +269,10 @@ struct strata_moe_layer_s {
     StackGraph graph;
     cudaEvent_t stage_ev[5];
     bool stage_on;
+    // n_tokens of the last call whose routing built the expert GEMMs' tile
+    // lists (strata_moe_route, or a forward on the tensor-core path); -1 after
+    // a call that did not (the one-launch decode layer, a stack)
+    int tiled_tokens;
 };
 
 static void stage_mark(strata_moe_layer L, int i, cudaStream_t st) {
@@ -333,6 +337,7 @@ extern "C" strata_status strata_moe_layer_create(const strata_moe_desc *desc, vo
     L->desc = *desc;
     L->shape = shape_of(desc);
     L->plan = plan;
+    L->tiled_tokens = -1;
     if (cudaGetDevice(&L->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) != cudaSuccess) {
         delete L;
@@ -438,6 +443,7 @@ static strata_status route_impl(strata_moe_layer L, const void *x, const float *
     strata_status s = router_impl(L, x, W, bias, L->ws.logits, T, st);
     if (s != STRATA_OK) return s;
     launch_route_large(L->ws, T, L->plan.max_tiles1, L->plan.max_tiles2, L->shape, st, x);
+    L->tiled_tokens = T;
     return check_launch("routing kernels");
 }
 
@@ -469,6 +475,7 @@ extern "C" strata_status strata_moe_forward(strata_moe_layer L, const void *x, c
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     stage_mark(L, 0, st);
     if (use_decode(L, T)) {
+        L->tiled_tokens = -1;
         stage_mark(L, 1, st);
         cudaError_t e = launch_decode_fused(L->ws, x, W, L->desc.router_bias, static_cast<const uint8_t *>(blob), y,
                                             (L->desc.flags & STRATA_ACCUMULATE) != 0, false, 0.f, T, L->shape,
@@ -515,6 +522,10 @@ extern "C" strata_status strata_moe_experts(strata_moe_layer L, const void *x, c
     if (!aligned16(x) || !aligned16(y)) return fail(STRATA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
     if (!aligned16(blob)) return fail(STRATA_ERR_BAD_BLOB, "expert blob must be 16-byte aligned");
     if (T == 0) return STRATA_OK;
+    if (L->tiled_tokens != T)
+        return fail(STRATA_ERR_INVALID_ARG,
+                    "strata_moe_experts needs the routing of a strata_moe_route call with n_tokens = %d on this handle "
+                    "(a forward of <= 16 tokens or a stack leaves none)", T);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     stage_mark(L, 1, st);
     s = experts_impl(L, x, blob, y, T, (L->desc.flags & STRATA_ACCUMULATE) != 0, st);
@@ -588,6 +599,7 @@ extern "C" strata_status strata_moe_stack_forward(strata_moe_layer L, int32_t n_
     }
     if (!aligned16(x)) return fail(STRATA_ERR_INVALID_ARG, "x_resid must be 16-byte aligned");
     if (T == 0 || n_layers == 0) return STRATA_OK;
+    L->tiled_tokens = -1;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int chunk = L->desc.max_tokens;
     const bool decode = T <= chunk && use_decode(L, T);
@@ -596,8 +608,9 @@ extern "C" strata_status strata_moe_stack_forward(strata_moe_layer L, int32_t n_
     if (!decode || cap != cudaStreamCaptureStatusNone) {
         for (int t0 = 0; t0 < T; t0 += chunk) {
             const int n = (T - t0) < chunk ? (T - t0) : chunk;
-            if ((s = stack_enqueue(L, n_layers, W, bias, blobs, x + (size_t)t0 * L->shape.d, n, eps, st)) != STRATA_OK)
-                return s;
+            s = stack_enqueue(L, n_layers, W, bias, blobs, x + (size_t)t0 * L->shape.d, n, eps, st);
+            L->tiled_tokens = -1;  // the layers' routing went to the workspace in turn
+            if (s != STRATA_OK) return s;
         }
         return STRATA_OK;
     }

@@ -190,8 +190,11 @@ strata_status strata_moe_route(strata_moe_layer layer, const void *x_bf16, const
                                int32_t n_tokens, strata_stream_t stream);
 
 /* Expert computation and combine for the routing of the last
- * strata_moe_route / strata_moe_forward call on this handle (same x and
- * n_tokens). */
+ * strata_moe_route call on this handle (same x and n_tokens), or of the last
+ * strata_moe_forward if that call took the tensor-core path (more than 16
+ * tokens, or STRATA_FORCE_PREFILL). Errors: INVALID_ARG when the handle's last
+ * routing call was not one of these, or had another n_tokens (a forward of
+ * <= 16 tokens on the one-launch path and a stack keep no tile lists). */
 strata_status strata_moe_experts(strata_moe_layer layer, const void *x_bf16, const void *expert_blob,
                                  float *y, int32_t n_tokens, strata_stream_t stream);
 

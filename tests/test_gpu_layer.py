@@ -341,3 +341,29 @@ def test_prefill_layer_8192_sampled_q4():
     routing, expert outputs on 48 sampled tokens."""
     e, nex = full_size_check(synth.WORKLOADS["prefill_q4"], 8192, 0, 48)
     print(f"4-bit prefill T=8192: max row err {e:.2e}, exempt {nex}")
+
+
+# ---------------------------------------------------------------- selection edge cases
+
+
+def _router(kind, E, d, seed):
+    W = synth.gen_router_w(seed, 0, E, d)
+    if kind == "zero":      # every logit 0: ties everywhere, all experts are candidates
+        return np.zeros_like(W)
+    if kind == "dup8":      # rows repeat with period 8: each logit value shared by E / 8 experts
+        return np.ascontiguousarray(W[np.arange(E) % 8])
+    return W
+
+
+@pytest.mark.parametrize("kind,E,k,T", [
+    ("zero", 128, 8, 2),     # more candidates than the selection keeps: exact one-warp pass
+    ("dup8", 64, 4, 3),      # exact ties among the top logits, resolved to the lower expert
+    ("dup8", 512, 10, 1),
+    ("plain", 64, 20, 4),    # k > 16: exact one-warp pass
+    ("plain", 32, 32, 1),    # k = E = 32
+])
+def test_selection_ties_and_fallbacks(kind, E, k, T):
+    d, f = 256, 128
+    h = HostLayer(d, f, E, k, T, seed=E + k + T, W=_router(kind, E, d, E + k))
+    err = check_full(h, run_layer(h, 0), exact_routing=False)
+    print(f"{kind} E={E} k={k} T={T}: max row err {err.max():.2e}")
