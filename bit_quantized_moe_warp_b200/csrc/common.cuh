@@ -216,6 +216,9 @@ STRATA_DEV float warp_sum(float v) {
 }
 
 STRATA_DEV float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// the same with the hardware exponential and a fast divide (a few fp32 ulp),
+// for products that are rounded to fp16 next
+STRATA_DEV float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Power-of-two scale of one token's activations for the fp16 operands: 1 when
 // the token's largest |x| is in [2^-4, 2^4] (the arithmetic is then the

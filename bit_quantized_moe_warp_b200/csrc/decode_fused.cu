@@ -412,6 +412,47 @@ __device__ __noinline__ void token_topk_exact(const float *logits, int t, int E,
     token_topk<16>(logits, t, E, k, sel_idx, sel_val);
 }
 
+// Adds the weighted outputs of one 16-row group x 8 token slots (an MMA C
+// fragment: lane (g, t) holds rows g, g+8 of slots 2t, 2t+1) into y with
+// 4-wide vector reductions. Lanes 4 apart share t; the four lanes of rows
+// 4p..4p+3 transpose their values (two butterfly exchanges), after which lane
+// 4p + v holds rows 8(v/2) + 4p .. +3 of slot 2t + (v%2), one reduction each:
+// a quarter of the scalar atomics, which meet every unit's adds to the same y.
+STRATA_DEV void add_rows4(float *y, int d, int row0, const float (&c)[4], int tokA, int tokB, float wA, float wB) {
+    const int lane = threadIdx.x & 31, g = lane >> 2;
+    float v[4] = {c[0] * wA, c[1] * wB, c[2] * wA, c[3] * wB};  // index 2h + e: row half h, slot parity e
+    const bool odd = g & 1, hi = g & 2;
+    {  // partner g ^ 1 (lane ^ 4): 2 x 2 transposes
+        const float r0 = __shfl_xor_sync(0xffffffffu, odd ? v[0] : v[1], 4);
+        const float r1 = __shfl_xor_sync(0xffffffffu, odd ? v[2] : v[3], 4);
+        if (odd) {
+            v[0] = r0;
+            v[2] = r1;
+        } else {
+            v[1] = r0;
+            v[3] = r1;
+        }
+    }
+    {  // partner g ^ 2 (lane ^ 8)
+        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[2], 8);
+        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? v[1] : v[3], 8);
+        if (hi) {
+            v[0] = r0;
+            v[1] = r1;
+        } else {
+            v[2] = r0;
+            v[3] = r1;
+        }
+    }
+    const int q = g & 3, tok = (q & 1) ? tokB : tokA;
+    if (tok >= 0) {
+        float *p = y + (size_t)tok * d + row0 + 8 * (q >> 1) + 4 * (g >> 2);
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                     "f"(v[3])
+                     : "memory");
+    }
+}
+
 template <int TT, int BITS>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedArgs a) {
     using CC = ChunkCfg<BITS>;
@@ -953,7 +994,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     // gs, us carry the token's scale s; h = silu(g) u is stored as h s^2
                     // (= silu(gs / s) us s), the down output is divided by s^2
                     const int tk = checked_index(ptok[eoff + slot], T, 0, status);
-                    h = silu_f(gs * xin[tk]) * us * xsc[tk];
+                    h = silu_fast(gs * xin[tk]) * us * xsc[tk];
                 }
                 hh[slot * kHStride + row] = __float2half_rn(h);
             }
@@ -992,31 +1033,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     if (!bad) {
                         const uint8_t *buf = bufs + (size_t)bi * kChunkBytes;
                         const int p0 = i * CC::kDownPanels, np = min(CC::kDownPanels, SLK - p0);
-                        for (int rgi = warp; rgi < np * 4; rgi += kFusedComputeWarps) {
-                            const int pan = rgi >> 2, r16 = 16 * (rgi & 3) + g;
-                            const TileRows<BITS> w = load_rows<BITS>(buf + (size_t)pan * CC::kTile, r16);
-                            float o[NT][4];
+                        // a warp takes DRG row groups of one panel at once: their rows
+                        // are loaded first and their MMA chains run interleaved
+                        constexpr int DRG = NT == 1 ? 4 : 2, TPP = 4 / DRG;
+                        for (int task = warp; task < np * TPP; task += kFusedComputeWarps) {
+                            const int pan = task / TPP, rg0 = (task % TPP) * DRG;
+                            TileRows<BITS> w[DRG];
 #pragma unroll
-                            for (int n = 0; n < NT; ++n)
+                            for (int r = 0; r < DRG; ++r)
+                                w[r] = load_rows<BITS>(buf + (size_t)pan * CC::kTile, 16 * (rg0 + r) + g);
+                            float o[DRG][NT][4];
 #pragma unroll
-                                for (int z = 0; z < 4; ++z) o[n][z] = 0.f;
-                            if (NT == 1 || nta == 1)
-                                down_rows<1, NT, ODD, BITS>(w, bf, zf, o);
-                            else
-                                down_rows<NT, NT, ODD, BITS>(w, bf, zf, o);
-                            const int row = (p0 + pan) * 64 + r16;
+                            for (int r = 0; r < DRG; ++r)
 #pragma unroll
-                            for (int n = 0; n < NT; ++n) {
-                                if (tokA[n] >= 0) {
-                                    float *yr = a.y + (size_t)tokA[n] * d + row;
-                                    atomicAdd(yr, wA[n] * o[n][0]);
-                                    atomicAdd(yr + 8, wA[n] * o[n][2]);
-                                }
-                                if (tokB[n] >= 0) {
-                                    float *yr = a.y + (size_t)tokB[n] * d + row;
-                                    atomicAdd(yr, wB[n] * o[n][1]);
-                                    atomicAdd(yr + 8, wB[n] * o[n][3]);
-                                }
+                                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                                    for (int z = 0; z < 4; ++z) o[r][n][z] = 0.f;
+#pragma unroll
+                            for (int r = 0; r < DRG; ++r) {
+                                if (NT == 1 || nta == 1)
+                                    down_rows<1, NT, ODD, BITS>(w[r], bf, zf, o[r]);
+                                else
+                                    down_rows<NT, NT, ODD, BITS>(w[r], bf, zf, o[r]);
+                            }
+#pragma unroll
+                            for (int r = 0; r < DRG; ++r) {
+                                const int row0 = (p0 + pan) * 64 + 16 * (rg0 + r);
+#pragma unroll
+                                for (int n = 0; n < NT; ++n)
+                                    add_rows4(a.y, d, row0, o[r][n], tokA[n], tokB[n], wA[n], wB[n]);
                             }
                         }
                     }
