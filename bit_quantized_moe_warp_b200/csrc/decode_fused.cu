@@ -30,12 +30,13 @@
 //            (contiguous in the blob), forms h = silu(g) * u for the slice in
 //            shared memory, then streams the down columns the slice feeds
 //            (contiguous too) and adds w * W_down[:, slice] h into y with
-//            fp32 atomics. One warp per CTA issues 1-D bulk copies of 40 KB
-//            chunks into a ring of shared-memory buffers and asks L2 for
-//            chunks other CTAs will copy later; 16 warps decode the 2-bit
-//            codes in registers straight into MMA fragments and multiply on
-//            the warp-level MMA (16 rows x 8 tokens x 16 columns, fp16 in,
-//            fp32 accumulate).
+//            4-wide fp32 vector reductions. One warp per CTA issues 1-D bulk
+//            copies of 40 KB chunks into a ring of shared-memory buffers and
+//            asks L2 for chunks other CTAs will copy later (and, while the
+//            lists are built, for one unit of the selection per CTA); 16
+//            warps decode the codes in registers straight into MMA fragments
+//            and multiply on the warp-level MMA (16 rows x 8 tokens x 16
+//            columns, fp16 in, fp32 accumulate).
 //
 // Exactness of the decode: a code c at mantissa bit p of an fp16 whose
 // exponent gives that bit the place value 1 is the exact value base_p + c
@@ -45,7 +46,8 @@
 // multiplying by the block's fp16 scale gives sum_k (c_k - 1.5) s x_k, up to
 // fp32 rounding. The 4-bit format (codes 0..15, offset 7.5) moves every
 // code to mantissa bits 4..7 (one shift per register at most), so all its
-// columns decode as 64 + c and Z = 71.5 sum_k x_k. Each token's x is staged as fp16(x * s) with s = 2^e putting
+// columns decode as 64 + c and Z = 71.5 sum_k x_k. Each token's x is staged
+// as fp16(x * s) with s = 2^e putting
 // its largest |x| in [1, 2): exact for every element within 2^-14 of that
 // largest, whatever the token's magnitude; the router sums and the gate/up
 // dot products carry s and are divided by it exactly. h, which grows as x^2,
@@ -457,7 +459,7 @@ template <int TT, int BITS>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedArgs a) {
     using CC = ChunkCfg<BITS>;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar;
+    __shared__ uint64_t full[kFusedMaxBuf], empty[kFusedMaxBuf], xbar, wbar, selbar;
     __shared__ int s_abort, s_nact;
     // per token: the power-of-two scale s of its staged x and 1 / s (exact);
     // per sorted pair: the routing weight / s^2 of its token
@@ -521,6 +523,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         }
         mbar_init(&xbar, 1);
         mbar_init(&wbar, 1);
+        mbar_init(&selbar, 1);  // the selection is known (phase 1)
         s_abort = 0;
         s_nact = 0;
         fence_mbar_init();
@@ -761,6 +764,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         if (warp < T && (!fast || ccnt[warp] > kCandMax))  // exact one-warp selection instead
             token_topk_exact(logits, warp, E, k, sel_idx + warp * k, sel_val + warp * k);
         compute_sync();
+        if (tid == 0) mbar_arrive(&selbar);
         if (warp < T) {  // renormalised softmax weights over the token's k selected (k <= 32)
             const float vmax = sel_val[warp * k];
             const float ex = lane < k ? expf(sel_val[warp * k + lane] - vmax) : 0.f;
@@ -834,6 +838,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             pslot[pos] = p % k;
             pw[pos] = sel_w[p];
             pws[pos] = sel_w[p] * xin[t] * xin[t];  // the down products carry s^2 of the token
+        }
+    } else if (!producer) {
+        if (tid == 0) mbar_arrive(&selbar);
+    } else if (lane == 0 && mbar_wait(&selbar, 0, status, &s_abort)) {
+        // Meanwhile the copy warp asks L2 for one (selected expert, 64-row
+        // slice) of the selection per CTA, about two microseconds before the
+        // per-expert lists exist and the ring copies start.
+        const int FP = f / 64, u = b;
+        if (u < T * k * FP) {
+            const int e = sel_idx[u / FP];
+            if (in_bounds(e, E, status)) {
+                const uint8_t *ebase = a.blob + (size_t)e * a.ebytes;
+                const int p = u % FP;
+                prefetch_l2(ebase + (size_t)p * a.xs.gu_panel, (uint32_t)(d / 64) * 2u * CC::kTile);
+                prefetch_l2(ebase + a.down_off + (size_t)p * a.xs.dn_slice, (uint32_t)(d / 64) * CC::kTile);
+            }
         }
     }
     __syncthreads();
@@ -980,7 +1000,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 }
             }
             compute_sync();
-            // ---- h = silu(g) * u for the slice's 64 rows (fp16) and its block constants
+            // ---- h = silu(g) * u for the slice's 64 rows (fp16) and its block
+            // constants: a warp's 32 items are one 32-row block of one slot
+            // (NS * 64 is a multiple of 512), reduced with shuffles
             for (int i = tid; i < NS * 64; i += 512) {
                 const int slot = i / 64, row = i % 64;
                 float h = 0.f;
@@ -996,10 +1018,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                     const int tk = checked_index(ptok[eoff + slot], T, 0, status);
                     h = silu_fast(gs * xin[tk]) * us * xsc[tk];
                 }
-                hh[slot * kHStride + row] = __float2half_rn(h);
+                const __half hv = __float2half_rn(h);
+                hh[slot * kHStride + row] = hv;
+                const float zc = warp_sum(column_weight<BITS>(row >> 1) * __half2float(hv));
+                if (lane == 0) hz[slot * 2 + (row >> 5)] = zc;
             }
-            compute_sync();
-            if (warp < NS) row_block_constants<BITS>(hh + warp * kHStride, 64, hz + warp * 2);
             compute_sync();
             // ---- down: y[token] += w * W_down[:, slice] h
             {
