@@ -844,9 +844,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
     } else if (lane == 0 && mbar_wait(&selbar, 0, status, &s_abort)) {
         // Meanwhile the copy warp asks L2 for one (selected expert, 64-row
         // slice) of the selection per CTA, about two microseconds before the
-        // per-expert lists exist and the ring copies start.
+        // per-expert lists exist and the ring copies start. Up to 4 tokens
+        // only: with more, the selection is several waves of units and these
+        // requests would queue ahead of the first ring copies.
         const int FP = f / 64, u = b;
-        if (u < T * k * FP) {
+        if (TT <= 4 && u < T * k * FP) {
             const int e = sel_idx[u / FP];
             if (in_bounds(e, E, status)) {
                 const uint8_t *ebase = a.blob + (size_t)e * a.ebytes;
@@ -1148,7 +1150,7 @@ constexpr int kFusedMinRing = 4;
 
 static FusedConfig fused_config(const Shape &s, int T, int max_smem) {
     FusedConfig c;
-    const int TT = T <= 1 ? 1 : T <= 4 ? 4 : 16;
+    const int TT = T <= 1 ? 1 : T <= 4 ? 4 : T <= 8 ? 8 : 16;
     const FusedSmem base = fused_plan(T, TT, s.d, s.E, s.k, 0);
     auto ring = [&](long long limit) {
         const long long room = limit - kFusedStaticSmem - (long long)base.total;
@@ -1175,13 +1177,14 @@ bool decode_fused_supported(const Shape &s, int T, int max_smem, int num_sms) {
 // (less L1), which slows the MMA loops (see kFusedSmemSoftCap). Kept per
 // device and instantiation; raised at layer creation, before any capture.
 static std::mutex g_limit_mutex;
-static int g_limit[64][6];
+static int g_limit[64][8];
 
 // the instantiation of a token count and code width
 using FusedKernel = void (*)(const FusedArgs);
 static FusedKernel kernel_of(int slot) {
-    static const FusedKernel k[6] = {k_decode_fused<1, 2>, k_decode_fused<4, 2>, k_decode_fused<16, 2>,
-                                     k_decode_fused<1, 4>, k_decode_fused<4, 4>, k_decode_fused<16, 4>};
+    static const FusedKernel k[8] = {k_decode_fused<1, 2>, k_decode_fused<4, 2>, k_decode_fused<8, 2>,
+                                     k_decode_fused<16, 2>, k_decode_fused<1, 4>, k_decode_fused<4, 4>,
+                                     k_decode_fused<8, 4>, k_decode_fused<16, 4>};
     return k[slot];
 }
 
@@ -1197,11 +1200,11 @@ static cudaError_t ensure_limit(int slot, int need) {
     return e;
 }
 
-static int slot_of(int T, int bits) { return (T <= 1 ? 0 : T <= 4 ? 1 : 2) + (bits == 4 ? 3 : 0); }
+static int slot_of(int T, int bits) { return (T <= 1 ? 0 : T <= 4 ? 1 : T <= 8 ? 2 : 3) + (bits == 4 ? 4 : 0); }
 
 cudaError_t init_fused_attributes(const Shape &s, int max_tokens, int max_smem, int num_sms) {
-    static const int tts[3] = {1, 4, 16};
-    for (int i = 0; i < 3; ++i) {
+    static const int tts[4] = {1, 4, 8, 16};
+    for (int i = 0; i < 4; ++i) {
         const int T = tts[i] < max_tokens ? tts[i] : max_tokens;
         if (slot_of(T, 2) != i || !decode_fused_supported(s, T, max_smem, num_sms)) continue;
         const cudaError_t e = ensure_limit(slot_of(T, s.bits), (int)fused_config(s, T, max_smem).smem);
