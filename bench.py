@@ -47,9 +47,10 @@ CSRC = os.path.join(ROOT, "bit_quantized_moe_warp_b200", "csrc")
 # When the sources differ the figure no longer describes the kernel and the
 # line reports traffic null.
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 19056128, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"),
-               "sha": "unrecorded"},
-    "prefill": {"bytes": 683305984, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "unrecorded"},
+    "decode": {"bytes": 19054848, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "46dca71ff63b0162"},
+    "decode_q4": {"bytes": 30854912, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "46dca71ff63b0162"},
+    "prefill": {"bytes": 683366912, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "d0da0b1f1847b92a"},
+    "prefill_q4": {"bytes": 871598336, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "d0da0b1f1847b92a"},
 }
 
 # library kernels per single-layer call: decode = the one-launch layer kernel;
@@ -97,7 +98,7 @@ def measured_traffic(name: str):
     None when there is none or the kernel's sources changed since."""
     m = MEASURED_TRAFFIC.get(name)
     if m is None:
-        return None, "no capture"
+        return None, "no capture of this shape"
     if sources_sha(m["sources"]) != m["sha"]:
         return None, "kernel changed since the last ncu capture"
     return m["bytes"], "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"
@@ -392,7 +393,7 @@ def decode_roofline(w, n_active, ms_per_launch, hbm, peak_src, launch_src):
     router = w.E * w.d * 4 + w.E * 4
     alg = decode_bytes(w, n_active)
     ach = sel / (ms_per_launch * 1e-3) / 1e9
-    traffic, tnote = measured_traffic("decode") if w.name in ("decode",) else (None, "no capture of this shape")
+    traffic, tnote = measured_traffic(w.name)
     return {"bound": "hbm", "kernel": "k_decode_fused (whole layer, one launch)", "achieved": ach, "peak": hbm,
             "unit": "GB/s", "frac": ach / hbm, "traffic": traffic, "traffic_note": tnote,
             "bytes_basis": "selected experts' packed weights (gate, up, down)",
@@ -410,7 +411,7 @@ def prefill_roofline(w, dom_ms, layer_ms, peak, peak_src, peak_kind):
     flops = w.T * w.k * 2 * 2 * w.d * w.f
     ach = flops / (dom_ms * 1e-3) / 1e12
     layer = expert_flops(w, w.T) / (layer_ms * 1e-3) / 1e12
-    traffic, tnote = measured_traffic("prefill") if w.name == "prefill" else (None, "no capture of this shape")
+    traffic, tnote = measured_traffic(w.name)
     return {"bound": "tensor", "kernel": f"k_expert_gemm<0, {w.bits}> (gate/up + SwiGLU)", "achieved": ach, "peak": peak,
             "unit": "TFLOP/s", "frac": ach / peak, "traffic": traffic, "traffic_note": tnote,
             "algorithmic_flops_per_launch": flops, "avg_launch_ms": dom_ms,
@@ -467,8 +468,8 @@ def measure(S, w, args, world, rank, local):
     block = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "q2+fp32" if T <= 16 else "q2+fp16->fp32",
-        "data": "synthetic (seeded; random-init 2-bit experts)",
+        "vs_baseline": None, "dtype": f"q{w.bits}+fp32" if T <= 16 else f"q{w.bits}+fp16->fp32",
+        "data": f"synthetic (seeded; random-init {w.bits}-bit experts)",
         "config": {"workload": w.name, "d_model": w.d, "d_ff": w.f, "n_experts": w.E, "top_k": w.k,
                    "tokens_per_step": T, "layers": w.layers, "routing": "zipf1.1" if w.zipf else "uniform",
                    "l2": (f"inputs larger than L2: {run.copies} seeded layer copies "
