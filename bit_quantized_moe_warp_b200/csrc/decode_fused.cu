@@ -551,21 +551,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         if (a.rms) {  // stack glue: bf16(RMSNorm) of the fp32 residual, one warp per token
             for (int t = warp; t < T; t += kFusedComputeWarps) {
                 const float4 *xr = reinterpret_cast<const float4 *>(static_cast<const float *>(a.x) + (size_t)t * d);
-                float ss = 0.f;
+                float ss = 0.f, am = 0.f;  // sum of squares; largest |x| (for the scale of the normalised row)
                 for (int c = lane; c < d / 4; c += 32) {
                     const float4 v = xr[c];
                     ss = fmaf(v.x, v.x, ss);
                     ss = fmaf(v.y, v.y, ss);
                     ss = fmaf(v.z, v.z, ss);
                     ss = fmaf(v.w, v.w, ss);
+                    am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
                 }
                 ss = warp_sum(ss);
                 const float inv = 1.0f / sqrtf(ss / (float)d + a.eps);
-                float am = 0.f;  // largest |x| of the token, for the scale of the normalised row
-                for (int c = lane; c < d / 4; c += 32) {
-                    const float4 v = xr[c];
-                    am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-                }
                 am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(am)));
                 const float sc = pow2_scale(am * inv);
                 if (lane == 0) {
