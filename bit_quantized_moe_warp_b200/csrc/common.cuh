@@ -215,9 +215,8 @@ STRATA_DEV float warp_sum(float v) {
     return v;
 }
 
-STRATA_DEV float silu_f(float g) { return g / (1.0f + expf(-g)); }
-// the same with the hardware exponential and a fast divide (a few fp32 ulp),
-// for products that are rounded to fp16 next
+// silu(g) = g / (1 + e^-g) with the hardware exponential and a fast divide (a
+// few fp32 ulp; both SwiGLU epilogues round the product to fp16 next)
 STRATA_DEV float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Power-of-two scale of one token's activations for the fp16 operands: 1 when

@@ -309,14 +309,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_expert_gemm(const __grid_co
                     if (unit) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            if (c0 + i < n) a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_f(g[i]) * u[i]);
+                            if (c0 + i < n) a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] = __float2half_rn(silu_fast(g[i]) * u[i]);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float sc = __shfl_sync(0xffffffffu, sl, i), inv = __shfl_sync(0xffffffffu, il, i);
                             if (c0 + i < n)
                                 a.H[(size_t)(p0 + c0 + i) * a.ldo + feat] =
-                                    __float2half_rn(silu_f(g[i] * inv) * u[i] * sc);
+                                    __float2half_rn(silu_fast(g[i] * inv) * u[i] * sc);
                         }
                     }
                 } else {
