@@ -47,10 +47,10 @@ CSRC = os.path.join(ROOT, "bit_quantized_moe_warp_b200", "csrc")
 # When the sources differ the figure no longer describes the kernel and the
 # line reports traffic null.
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 19054848, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "46dca71ff63b0162"},
-    "decode_q4": {"bytes": 30854912, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "46dca71ff63b0162"},
-    "prefill": {"bytes": 683366912, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "d0da0b1f1847b92a"},
-    "prefill_q4": {"bytes": 871598336, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "d0da0b1f1847b92a"},
+    "decode": {"bytes": 19052288, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "894c3391b0f04cf9"},
+    "decode_q4": {"bytes": 30853632, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "894c3391b0f04cf9"},
+    "prefill": {"bytes": 683609344, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "6cbc1f503f5c52df"},
+    "prefill_q4": {"bytes": 872128256, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "6cbc1f503f5c52df"},
 }
 
 # library kernels per single-layer call: decode = the one-launch layer kernel;
