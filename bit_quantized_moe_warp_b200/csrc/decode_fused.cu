@@ -761,11 +761,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
             token_topk_exact(logits, warp, E, k, sel_idx + warp * k, sel_val + warp * k);
         compute_sync();
         if (tid == 0) mbar_arrive(&selbar);
-        if (warp < T) {  // renormalised softmax weights over the token's k selected (k <= 32)
-            const float vmax = sel_val[warp * k];
-            const float ex = lane < k ? expf(sel_val[warp * k + lane] - vmax) : 0.f;
+        // renormalised softmax weights over token t's k selected (k <= 32), on
+        // warp 15 - t: warp 0 has just released the selection to the copy warp,
+        // and its shuffles measured 0.7 us slower there
+        if (kFusedComputeWarps - 1 - warp < T) {
+            const int t = kFusedComputeWarps - 1 - warp;
+            const float vmax = sel_val[t * k];
+            const float ex = lane < k ? expf(sel_val[t * k + lane] - vmax) : 0.f;
             const float den = warp_sum(ex);
-            if (lane < k) sel_w[warp * k + lane] = ex / den;
+            if (lane < k) sel_w[t * k + lane] = ex / den;
         }
         for (int i = tid; i < T * k; i += 512)
             if (in_bounds(sel_idx[i], E, status)) atomicOr(&mask[sel_idx[i]], 1u << (i / k));
