@@ -493,49 +493,130 @@ def measure(S, w, args, world, rank, local):
 def end_to_end(run, steps, world):
     """The same metric through the public API with host buffers: every step
     copies that step's x from pinned host memory, runs the layer (or stack)
-    through the C ABI and reads y back into pinned host memory."""
+    through the C ABI and reads y back into pinned host memory. Single layers
+    of more than 16 tokens run as a two-buffer pipeline, as a serving loop
+    does: the input and output copies (own streams, ordered by events) overlap
+    the neighbouring steps' layer calls. At 16 tokens or fewer the copies are
+    a few KB and the extra stream and event calls cost more host time than
+    they hide, so the steps run on one stream."""
     import torch
     S, w, T = run.S, run.w, run.T
     dev = run.dev
+    n = max(8, min(steps, 2048 if T <= 16 else 8)) if not run.stacked else 2
+    h2d = T * w.d * (4 if run.stacked else 2)
+    d2h = T * w.d * 4
+    if not run.stacked and T <= 16:
+        xh = torch.empty((64, T, w.d), dtype=torch.bfloat16).pin_memory()
+        xh.copy_(torch.randn(64, T, w.d).to(torch.bfloat16))
+        outh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
+        xd = torch.empty((T, w.d), dtype=torch.bfloat16, device=dev)
+        yd = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream().cuda_stream
+        args = [(run.handles[c].handle, run.layers[c].W.data_ptr(), run.layers[c].blob.data_ptr())
+                for c in range(run.copies)]
+        xp, yp = xd.data_ptr(), yd.data_ptr()
+        xhs = [xh[i] for i in range(64)]
+
+        def one(i):
+            h, Wp, bp = args[i % run.copies]
+            xd.copy_(xhs[i % 64], non_blocking=True)
+            S.strata_moe_forward(h, xp, Wp, bp, yp, T, st)
+            outh.copy_(yd, non_blocking=True)
+
+        for i in range(3):
+            one(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            one(i)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = dist_max(e0.elapsed_time(e1), world)
+        return {"value": T * n * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n,
+                "note": "every step: pinned host x -> device, forward through the C ABI (Python binding), "
+                        "y -> pinned host, on one stream"}
     if run.stacked:
         xh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
         xh.copy_(torch.randn(T, w.d))
         outh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
         xd = torch.empty((T, w.d), dtype=torch.float32, device=dev)
-    else:
-        xh = torch.empty((64, T, w.d), dtype=torch.bfloat16).pin_memory()
-        xh.copy_(torch.randn(64, T, w.d).to(torch.bfloat16))
-        outh = torch.empty((T, w.d), dtype=torch.float32).pin_memory()
-        xd = torch.empty((T, w.d), dtype=torch.bfloat16, device=dev)
-    yd = torch.zeros((T, w.d), dtype=torch.float32, device=dev)
-    n = max(8, min(steps, 2048 if T <= 16 else 8)) if not run.stacked else 2
 
-    def one(i):
-        if run.stacked:
+        def one(i):
             xd.copy_(xh, non_blocking=True)
             run.handle.stack_forward([l.W for l in run.layers], [l.bias for l in run.layers] if w.zipf else None,
                                      [l.blob for l in run.layers], xd, T, 1e-6)
             outh.copy_(xd, non_blocking=True)
-        else:
-            c = i % run.copies
-            xd.copy_(xh[i % 64], non_blocking=True)
-            run.handles[c].forward(xd, run.layers[c].W, run.layers[c].blob, yd, T)
-            outh.copy_(yd, non_blocking=True)
 
-    for i in range(3):
+        for i in range(3):
+            one(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            one(i)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = dist_max(e0.elapsed_time(e1), world)
+        return {"value": T * n * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n,
+                "note": "pinned host x -> device, stack through the C ABI (Python binding), x -> pinned host"}
+
+    nx = 2
+    xh = torch.empty((nx, T, w.d), dtype=torch.bfloat16).pin_memory()
+    xh.copy_(torch.randn(nx, T, w.d).to(torch.bfloat16))
+    outh = [torch.empty((T, w.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+    xd = [torch.empty((T, w.d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    yd = [torch.zeros((T, w.d), dtype=torch.float32, device=dev) for _ in range(2)]
+    s_c = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]   # x buffer b filled
+    ev_k = [torch.cuda.Event() for _ in range(2)]    # layer call on buffer b done
+    ev_out = [torch.cuda.Event() for _ in range(2)]  # y buffer b copied out
+    st = s_c.cuda_stream
+    # the layer call with plain device addresses and the stream handle
+    args = [(run.handles[c].handle, run.layers[c].W.data_ptr(), run.layers[c].blob.data_ptr())
+            for c in range(run.copies)]
+    xp, yp = [t.data_ptr() for t in xd], [t.data_ptr() for t in yd]
+    xhs = [xh[i] for i in range(nx)]
+
+    def one(i):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(ev_k[b])       # the call two steps back has read xd[b]
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(xhs[i % nx], non_blocking=True)
+        ev_in[b].record(s_in)
+        s_c.wait_event(ev_in[b])
+        if i >= 2:
+            s_c.wait_event(ev_out[b])      # yd[b] of two steps back is on the host
+        h, Wp, bp = args[i % run.copies]
+        S.strata_moe_forward(h, xp[b], Wp, bp, yp[b], T, st)
+        ev_k[b].record(s_c)
+        s_out.wait_event(ev_k[b])
+        with torch.cuda.stream(s_out):
+            outh[b].copy_(yd[b], non_blocking=True)
+        ev_out[b].record(s_out)
+
+    for i in range(4):
         one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s_c)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
     for i in range(n):
         one(i)
-    e1.record()
+    s_c.wait_stream(s_out)
+    e1.record(s_c)
     torch.cuda.synchronize()
     ms = dist_max(e0.elapsed_time(e1), world)
-    h2d = T * w.d * (4 if run.stacked else 2)
     return {"value": T * n * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": T * w.d * 4, "steps": n,
-            "note": "pinned host x -> device, forward through the C ABI (Python binding), y -> pinned host"}
+            "d2h_bytes_per_step": d2h, "steps": n,
+            "note": "every step: pinned host x -> device, forward through the C ABI (Python binding), "
+                    "y -> pinned host; two buffers, copies on their own streams overlapping the neighbouring "
+                    "steps' layer calls"}
 
 
 # ---------------------------------------------------------------- CPU oracle
