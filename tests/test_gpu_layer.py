@@ -310,6 +310,7 @@ Q4_SHAPES = [
     # d, f, E, k, T, zipf, flags
     (256, 128, 16, 4, 1, False, 0),
     (384, 256, 64, 10, 16, True, 0),
+    (256, 128, 32, 8, 6, True, 0),     # the 8-token instantiation
     (256, 256, 64, 10, 17, True, 0),   # first prefill size
     (512, 128, 64, 4, 130, True, 0),   # ragged tiles
     (128, 256, 16, 2, 1000, True, 0),  # several 128/256-token tiles per expert
