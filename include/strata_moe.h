@@ -49,7 +49,7 @@ typedef struct CUstream_st *strata_stream_t;
 typedef enum {
     STRATA_OK = 0,
     STRATA_ERR_INVALID_ARG = -1,    /* bad pointer, size, alignment or desc */
-    STRATA_ERR_UNSUPPORTED = -2,    /* shape or flag this build does not run */
+    STRATA_ERR_UNSUPPORTED = -2,    /* shape, format or flag the library does not run */
     STRATA_ERR_CUDA = -3,           /* a CUDA runtime call failed */
     STRATA_ERR_OOM = -4,            /* workspace allocation failed */
     STRATA_ERR_TOO_MANY_TOKENS = -5,/* n_tokens > max_tokens (layer calls) */
