@@ -638,24 +638,26 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
                 for (int i = 0; i < 4; ++i) {
                     if (128 * i + 4 * lane < ncol) {
                         const float4 wv = *reinterpret_cast<const float4 *>(wrow + cbase + c0 + 128 * i + 4 * lane);
+                        // slots past the last token read the zero row: no branch
+                        // between the loads, so they are all in flight at once
 #pragma unroll
                         for (int t = 0; t < TT; ++t) {
-                            if (t < T) {
-                                const uint2 xv =
-                                    *reinterpret_cast<const uint2 *>(xh + (size_t)t * dpx + cbase + c0 + 128 * i + 4 * lane);
-                                const float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.x));
-                                const float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.y));
-                                acc[t] = fmaf(wv.x, x01.x, acc[t]);
-                                acc[t] = fmaf(wv.y, x01.y, acc[t]);
-                                acc[t] = fmaf(wv.z, x23.x, acc[t]);
-                                acc[t] = fmaf(wv.w, x23.y, acc[t]);
-                            }
+                            const int tr = t < T ? t : T;
+                            const uint2 xv =
+                                *reinterpret_cast<const uint2 *>(xh + (size_t)tr * dpx + cbase + c0 + 128 * i + 4 * lane);
+                            const float2 x01 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.x));
+                            const float2 x23 = __half22float2(*reinterpret_cast<const __half2 *>(&xv.y));
+                            acc[t] = fmaf(wv.x, x01.x, acc[t]);
+                            acc[t] = fmaf(wv.y, x01.y, acc[t]);
+                            acc[t] = fmaf(wv.z, x23.x, acc[t]);
+                            acc[t] = fmaf(wv.w, x23.y, acc[t]);
                         }
                     }
                 }
             }
 #pragma unroll
-            for (int t = 0; t < TT; ++t) acc[t] = warp_sum(acc[t]);
+            for (int t = 0; t < TT; ++t)
+                if (t < T) acc[t] = warp_sum(acc[t]);
             if (lane == 0)
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
@@ -698,10 +700,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_decode_fused(const FusedAr
         uint32_t key[TT];
         if (fast && t < T) {
             const float *row = logits + (size_t)t * E;
+            // every lane loads (past a group's end it re-reads the group's last
+            // logit), so the TT loads are in flight at once; then the keys
+            float v[TT];
 #pragma unroll
             for (int r = 0; r < TT; ++r) {
                 const int q = g * TT + r, lo = q * E / 16, hi = (q + 1) * E / 16;
-                key[r] = lo + lane < hi ? ordered_key(__ldcg(row + lo + lane)) : 0u;  // 0: below every real key
+                v[r] = __ldcg(row + (lo + lane < hi ? lo + lane : (hi > lo ? hi - 1 : 0)));
+            }
+#pragma unroll
+            for (int r = 0; r < TT; ++r) {
+                const int q = g * TT + r, lo = q * E / 16, hi = (q + 1) * E / 16;
+                key[r] = lo + lane < hi ? ordered_key(v[r]) : 0u;  // 0: below every real key
             }
 #pragma unroll
             for (int r = 0; r < TT; ++r) {
