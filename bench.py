@@ -47,8 +47,8 @@ CSRC = os.path.join(ROOT, "bit_quantized_moe_warp_b200", "csrc")
 # When the sources differ the figure no longer describes the kernel and the
 # line reports traffic null.
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 19053568, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "78f5e25ba9ee8df5"},
-    "decode_q4": {"bytes": 30854400, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "78f5e25ba9ee8df5"},
+    "decode": {"bytes": 19053312, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "41f61124a013c376"},
+    "decode_q4": {"bytes": 30853632, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "41f61124a013c376"},
     "prefill": {"bytes": 683609344, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "6cbc1f503f5c52df"},
     "prefill_q4": {"bytes": 872128256, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "6cbc1f503f5c52df"},
 }
