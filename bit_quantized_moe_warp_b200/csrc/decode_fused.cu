@@ -4,9 +4,11 @@
 // A decode step verifies 1 + up to 3 draft tokens in one 48-layer pass
 // ("Strata：把 125B 大模型塞进 12GB 显卡，24,576 个专家在内存与 SSD 之间流动",
 // 再快一截：先猜再验的投机解码); every token uses 10 experts (核心思路). At these
-// sizes the layer is bound by the bytes of the selected experts' 2-bit
-// weights and by the latency of the steps before them, so the kernel pays
-// the routing latency once and then keeps the weight stream busy:
+// sizes the layer is bound by the bytes of the selected experts' 2-bit (or
+// 4-bit) weights and by the latency of the steps before them, so the kernel
+// pays the routing latency once and then keeps the weight stream busy. It is
+// launched as a programmatic dependent of the previous kernel on the stream
+// and waits for it (griddepcontrol.wait) before touching memory.
 //
 //   phase 0  one warp per CTA starts bulk copies of x and of the CTA's slice
 //            of router rows (the bias comes by cp.async); the other warps
@@ -31,7 +33,8 @@
 //            shared memory, then streams the down columns the slice feeds
 //            (contiguous too) and adds w * W_down[:, slice] h into y with
 //            4-wide fp32 vector reductions. One warp per CTA issues 1-D bulk
-//            copies of 40 KB chunks into a ring of shared-memory buffers and
+//            copies of 40 KB chunks (36 KB of 4-bit tiles) into a ring of
+//            shared-memory buffers and
 //            asks L2 for chunks other CTAs will copy later (and, while the
 //            lists are built, for one unit of the selection per CTA); 16
 //            warps decode the codes in registers straight into MMA fragments
@@ -47,12 +50,11 @@
 // fp32 rounding. The 4-bit format (codes 0..15, offset 7.5) moves every
 // code to mantissa bits 4..7 (one shift per register at most), so all its
 // columns decode as 64 + c and Z = 71.5 sum_k x_k. Each token's x is staged
-// as fp16(x * s) with s = 2^e putting
-// its largest |x| in [1, 2): exact for every element within 2^-14 of that
-// largest, whatever the token's magnitude; the router sums and the gate/up
-// dot products carry s and are divided by it exactly. h, which grows as x^2,
-// is rounded to fp16 as h * s^2 (relative error <= 2^-11) and the down output
-// is divided by s^2.
+// as fp16(x * s) with s = 2^e putting its largest |x| in [1, 2): exact for
+// every element within 2^-14 of that largest, whatever the token's
+// magnitude; the router sums and the gate/up dot products carry s and are
+// divided by it exactly. h, which grows as x^2, is rounded to fp16 as h * s^2
+// (relative error <= 2^-11) and the down output is divided by s^2.
 //
 // Every wait (grid barrier, copy barrier) is time-bounded; on expiry the
 // kernel records a timeout in the status word and unwinds. Decisions to stop
