@@ -92,3 +92,15 @@ def test_traffic_is_dropped_when_kernel_sources_change():
         assert bench.measured_traffic("decode")[0] is None
     finally:
         m["sha"] = saved
+
+
+def test_traffic_guard_ignores_comments_only(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("// header\n__global__ void k(int *p) {\n    p[0] = 1;  // store\n}\n")
+    monkeypatch.setattr(bench, "CSRC", str(tmp_path))
+    h0 = bench.sources_sha(("k.cu",))
+    src.write_text("/* a longer\n   header */\n__global__ void k(int *p) {\n\n    p[0] = 1;  // the store\n}\n")
+    assert bench.sources_sha(("k.cu",)) == h0
+    src.write_text("// header\n__global__ void k(int *p) {\n    p[0] = 2;  // store\n}\n")
+    assert bench.sources_sha(("k.cu",)) != h0
+
