@@ -64,6 +64,19 @@ def _bind(lib):
     lib.oracle_moe_layer.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.oracle_rmsnorm_bf16.argtypes = [I, P, ctypes.c_double, P]
     lib.oracle_residual_add_f32.argtypes = [I, P, P]
+    lib.oracle_float_to_fp16.restype = ctypes.c_uint16
+    lib.oracle_float_to_fp16.argtypes = [ctypes.c_float]
+    lib.oracle_hadamard_sign.restype = I
+    lib.oracle_hadamard_sign.argtypes = [I, I]
+    L = ctypes.c_long
+    lib.oracle_fwht_f32.argtypes = [I, P]
+    lib.oracle_kv4_quantize_block.argtypes = [P, P, P]
+    lib.oracle_kv4_encode.argtypes = [L, I, P, P, P]
+    lib.oracle_kv4_decode.argtypes = [L, I, P, P, P]
+    lib.oracle_round_bf16_array.argtypes = [L, P, P]
+    for fn in ("oracle_fwht_f32", "oracle_kv4_quantize_block", "oracle_kv4_encode", "oracle_kv4_decode",
+               "oracle_round_bf16_array"):
+        getattr(lib, fn).restype = None
     for fn in ("oracle_dequant", "oracle_unpack_q2_tiled", "oracle_unpack_q4_tiled", "oracle_router_logits",
                "oracle_topk_softmax", "oracle_expert_lists", "oracle_expert_ffn",
                "oracle_moe_layer", "oracle_rmsnorm_bf16", "oracle_residual_add_f32"):
@@ -246,6 +259,61 @@ def residual_add_f32(x_f32, y):
     y = _c(y, np.float64)
     load().oracle_residual_add_f32(x.size, _p(x), _p(y))
     return x
+
+
+# ----------------------------------------------------------------------------
+# 4-bit Hadamard-rotated KV-cache codec
+
+
+def float_to_fp16(v):
+    """fp32 values -> fp16 bit patterns (round to nearest even)."""
+    lib = load()
+    return np.array([lib.oracle_float_to_fp16(float(x)) for x in np.ravel(np.asarray(v, dtype=np.float32))],
+                    dtype=np.uint16).reshape(np.shape(v))
+
+
+def hadamard_sign(i: int, j: int) -> int:
+    return load().oracle_hadamard_sign(int(i), int(j))
+
+
+def fwht_f32(v):
+    """Unnormalised Walsh-Hadamard transform of one fp32 vector (fp32 steps)."""
+    v = np.array(v, dtype=np.float32)
+    load().oracle_fwht_f32(v.size, _p(v))
+    return v
+
+
+def kv4_quantize_block(y):
+    """One 32-value block -> (codes uint8[32] in 1..15, fp16 scale bits)."""
+    y = _c(y, np.float32)
+    assert y.size == 32
+    code = np.empty(32, dtype=np.uint8)
+    sb = np.zeros(1, dtype=np.uint16)
+    load().oracle_kv4_quantize_block(_p(y), _p(code), _p(sb))
+    return code, int(sb[0])
+
+
+def kv4_encode(x_bf16):
+    """bf16 rows [rows, D] -> (codes uint8 [rows, D/2], scales fp16 bits uint16 [rows, D/32])."""
+    x = _c(x_bf16, np.uint16)
+    rows, D = x.shape
+    codes = np.empty((rows, D // 2), dtype=np.uint8)
+    scales = np.empty((rows, D // 32), dtype=np.uint16)
+    load().oracle_kv4_encode(rows, D, _p(x), _p(codes), _p(scales))
+    return codes, scales
+
+
+def kv4_decode(codes, scales):
+    """(codes, scales) -> (exact values as double [rows, D], their bf16 bits)."""
+    codes = _c(codes, np.uint8)
+    sc = _c(np.asarray(scales).view(np.uint16), np.uint16)
+    rows, D = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((rows, D), dtype=np.float64)
+    bits = np.empty((rows, D), dtype=np.uint16)
+    lib = load()
+    lib.oracle_kv4_decode(rows, D, _p(codes), _p(sc), _p(out))
+    lib.oracle_round_bf16_array(out.size, _p(out), _p(bits))
+    return out, bits
 
 
 # ----------------------------------------------------------------------------

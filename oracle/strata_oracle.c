@@ -1,6 +1,7 @@
 /*
  * strata_oracle.c -- plain, slow, single-threaded CPU oracle of the
- * routed-expert MoE layer with 2-bit block-quantised experts.
+ * routed-expert MoE layer with 2-bit block-quantised experts, and of the
+ * 4-bit Hadamard-rotated KV-cache codec.
  *
  * TEST INFRASTRUCTURE ONLY. Nothing in the library calls this file; only the
  * tests, the smoke check and the benchmark's CPU-baseline leg load it. It
@@ -35,6 +36,22 @@
  *    block format here is the same rule with 4-bit codes: c in {0..15}
  *    meaning (c - 7.5) * scale, one fp16 scale per 32 weights. In general a
  *    b-bit code means c - (2^b - 1) / 2, centred on zero.
+ *
+ *  - The optional 4-bit KV cache ("Strata：把 125B 大模型塞进 12GB 显卡…",
+ *    长上下文 section; its 代码结构 section lists q4/q8 KV kernels): one
+ *    Hadamard rotation of each cached key/value vector, then 4-bit rounding,
+ *    halving the memory of the default 8-bit cache. The pages give neither
+ *    the rotation's normalisation nor the rounding grid. Read here: the
+ *    orthonormal Walsh-Hadamard rotation y = H x / sqrt(D) of each head_dim-D
+ *    row (D a power of two, H the Sylvester matrix, H[i][j] =
+ *    (-1)^popcount(i & j)); 32-value blocks with one fp16 scale
+ *    s = fp16(absmax / 7) (saturated at 65504); q = round-half-even(y / s)
+ *    clamped to [-7, 7], stored as the nibble q + 8; decoding inverts:
+ *    x = H ((c - 8) s) / sqrt(D), rounded to bf16. Because the codes are
+ *    integers decided by floating point, the encoder computes in fp32 in a
+ *    fixed order (butterfly stages of stride 1, 2, ..., D/2, then the
+ *    product by fp32(1/sqrt(D)), then the block quantiser); the decoder, whose
+ *    output is a float, is the fp64 matrix-vector definition.
  *
  * Readings taken where the pages are silent (each also listed in the design
  * notes): the top-k order key is the logit rounded to fp32 (the precision the
@@ -356,4 +373,130 @@ void oracle_residual_add_f32(int n, float *x, const double *y)
 {
     for (int i = 0; i < n; ++i)
         x[i] = (float)((double)x[i] + y[i]);
+}
+
+/* ------------------------------------------- 4-bit rotated KV-cache codec */
+
+/* fp32 -> IEEE binary16 bits, one rounding to nearest, ties to even; values
+ * beyond the largest finite half become infinity. */
+uint16_t oracle_float_to_fp16(float f)
+{
+    uint16_t sign = signbit(f) ? 0x8000 : 0x0000;
+    double v = fabs((double)f);
+    if (v == 0.0)
+        return sign;
+    int e;
+    frexp(v, &e); /* v = m 2^e, m in [0.5, 1) */
+    int qe = e - 11; /* 11 significant bits: quantum 2^(e-11) */
+    if (qe < -24)
+        qe = -24; /* subnormal range: fixed quantum 2^-24 */
+    double n = nearbyint(ldexp(v, -qe)); /* quanta, ties to even */
+    if (n >= 2048.0) { /* rounded up into the next binade */
+        n /= 2.0;
+        qe += 1;
+    }
+    if (n < 1024.0) /* subnormal (qe == -24) */
+        return sign | (uint16_t)n;
+    if (qe + 25 >= 31)
+        return sign | 0x7c00;
+    return sign | (uint16_t)(((qe + 25) << 10) | ((int)n - 1024));
+}
+
+/* Sylvester-Hadamard entry H[i][j] = (-1)^popcount(i & j) */
+int oracle_hadamard_sign(int i, int j)
+{
+    int p = 0;
+    for (unsigned m = (unsigned)(i & j); m; m >>= 1)
+        p ^= (int)(m & 1u);
+    return p ? -1 : 1;
+}
+
+/* Unnormalised Walsh-Hadamard transform of v[0..D) in place, in fp32: for
+ * stride h = 1, 2, ..., D/2 every pair (i, i + h) with bit h of i clear
+ * becomes (v_i + v_{i+h}, v_i - v_{i+h}). Exact arithmetic gives H v. */
+void oracle_fwht_f32(int D, float *v)
+{
+    for (int h = 1; h < D; h *= 2)
+        for (int i = 0; i < D; ++i)
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+/* One 32-value block: s = fp16(min(absmax / 7, 65504)), all in fp32;
+ * q_i = clamp(rint(y_i / s), -7, 7) (q = 0 when s is zero); code q_i + 8. */
+void oracle_kv4_quantize_block(const float *y, uint8_t *code, uint16_t *scale_bits)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i)
+        if (fabsf(y[i]) > amax)
+            amax = fabsf(y[i]);
+    float t = amax / 7.0f;
+    if (t > 65504.0f)
+        t = 65504.0f;
+    uint16_t sb = oracle_float_to_fp16(t);
+    float s = (float)oracle_fp16_to_double(sb);
+    for (int i = 0; i < 32; ++i) {
+        int q = 0;
+        if (s > 0.0f) {
+            float r = rintf(y[i] / s); /* default rounding mode: ties to even */
+            q = r > 7.0f ? 7 : (r < -7.0f ? -7 : (int)r);
+        }
+        code[i] = (uint8_t)(q + 8);
+    }
+    *scale_bits = sb;
+}
+
+/* Encoder. x: bf16 bits [rows x D]; codes: [rows x D/2] bytes, element 2j in
+ * the low nibble of byte j and 2j+1 in the high nibble; scales: fp16 bits
+ * [rows x D/32]. y = fp32(FWHT(x) * fp32(1/sqrt(D))), then the block rule. */
+void oracle_kv4_encode(long rows, int D, const uint16_t *x, uint8_t *codes, uint16_t *scales)
+{
+    float r = (float)(1.0 / sqrt((double)D));
+    float *y = malloc((size_t)D * sizeof *y);
+    uint8_t q[32];
+    for (long row = 0; row < rows; ++row) {
+        for (int i = 0; i < D; ++i)
+            y[i] = (float)oracle_bf16_to_double(x[(size_t)row * D + i]);
+        oracle_fwht_f32(D, y);
+        for (int i = 0; i < D; ++i)
+            y[i] = y[i] * r;
+        for (int b = 0; b < D / 32; ++b) {
+            oracle_kv4_quantize_block(y + 32 * b, q, &scales[(size_t)row * (D / 32) + b]);
+            for (int j = 0; j < 16; ++j)
+                codes[(size_t)row * (D / 2) + 16 * b + j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+        }
+    }
+    free(y);
+}
+
+/* Decoder, the definition in double: y_i = (c_i - 8) * s_(i/32),
+ * x_j = sum_i H[j][i] y_i / sqrt(D). out: [rows x D] exact-as-double values
+ * (the caller rounds them to bf16). */
+void oracle_kv4_decode(long rows, int D, const uint8_t *codes, const uint16_t *scales, double *out)
+{
+    double inv = 1.0 / sqrt((double)D);
+    double *y = malloc((size_t)D * sizeof *y);
+    for (long row = 0; row < rows; ++row) {
+        for (int i = 0; i < D; ++i) {
+            int c = (codes[(size_t)row * (D / 2) + i / 2] >> (4 * (i % 2))) & 15;
+            y[i] = (c - 8) * oracle_fp16_to_double(scales[(size_t)row * (D / 32) + i / 32]);
+        }
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i)
+                acc += oracle_hadamard_sign(j, i) * y[i];
+            out[(size_t)row * D + j] = acc * inv;
+        }
+    }
+    free(y);
+}
+
+/* out[i] = bf16(v[i]) for a whole array (one rounding each) */
+void oracle_round_bf16_array(long n, const double *v, uint16_t *out)
+{
+    for (long i = 0; i < n; ++i)
+        out[i] = oracle_double_to_bf16(v[i]);
 }

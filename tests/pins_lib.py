@@ -438,4 +438,208 @@ def check_residual_add():
     assert np.array_equal(got, (x.astype(np.float64) + y).astype(np.float32))
 
 
+# ------------------------------------------- 4-bit rotated KV-cache codec
+
+
+def hadamard(D: int) -> np.ndarray:
+    """Sylvester Hadamard matrix from scipy (a library routine, not the oracle)."""
+    import scipy.linalg
+    return scipy.linalg.hadamard(D).astype(np.float64)
+
+
+def fp16_rne_exact(v: float) -> int:
+    """IEEE binary16 round-to-nearest-even of a double, in exact rationals."""
+    if v == 0.0:
+        return 0x8000 if math.copysign(1.0, v) < 0 else 0
+    m, e = math.frexp(abs(v))
+    qe = max(e - 11, -24)
+    n = round(Fraction(abs(v)) / Fraction(2) ** qe)
+    return int(np.array([float(n * Fraction(2) ** qe) * (1 if v > 0 else -1)], dtype=np.float64)
+               .astype(np.float16).view(np.uint16)[0])
+
+
+def bf16_bits(v) -> np.ndarray:
+    return (np.asarray(v, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def kv_rows(seed: int, rows: int, D: int) -> np.ndarray:
+    """bf16 rows, N(0,1) with a few large outliers per row (cached keys and
+    values carry such channels)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, D)).astype(np.float32)
+    big = rng.integers(0, D, (rows, 2))
+    for r in range(rows):
+        x[r, big[r]] *= 20.0
+    return bf16_bits(x)
+
+
+def load_kv_example():
+    cases = []
+    with open(os.path.join(GOLD, "kv4_example.txt")) as fh:
+        for line in fh:
+            t = line.split("#", 1)[0].split()
+            if t:
+                cases.append((t[0], dict(kv.split("=", 1) for kv in t[1:])))
+    return cases
+
+
+def check_fp16_encode():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        rng.standard_normal(3000) * 10.0 ** rng.integers(-9, 5, 3000),
+        1 + (2 * rng.integers(0, 1024, 300) + 1) * 2.0 ** -11,  # ties in [1, 2)
+        (2 * rng.integers(0, 512, 300) + 1) * 2.0 ** -25,  # ties in the subnormal range
+        [65504.0, 65519.0, 65520.0, 2.0 ** -14, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 0.0, -0.0]])
+    vals = vals.astype(np.float32)
+    got = O.float_to_fp16(vals)
+    with np.errstate(over="ignore"):
+        lib = vals.astype(np.float16).view(np.uint16)  # numpy's IEEE conversion
+    assert np.array_equal(got, lib), "fp16 rounding differs from IEEE round-to-nearest-even"
+    for v in (1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 2.0 ** -25, 3 * 2.0 ** -25, 0.017857142857142856):
+        assert int(O.float_to_fp16([v])[0]) == fp16_rne_exact(float(np.float32(v))), v
+
+
+def check_kv4_fwht_is_hadamard():
+    rng = np.random.default_rng(12)
+    for D in (32, 64, 128, 256):
+        H = hadamard(D)
+        for i in (0, 1, D // 2 + 3, D - 1):
+            for j in (0, 2, D // 3, D - 1):
+                assert O.hadamard_sign(i, j) == H[i, j], (D, i, j)
+        v = rng.integers(-100, 101, D).astype(np.float32)  # exact in fp32 throughout
+        assert np.array_equal(O.fwht_f32(v).astype(np.float64), H @ v.astype(np.float64)), D
+        v = (rng.standard_normal(D) * 10.0 ** rng.integers(-3, 3, D)).astype(np.float32)
+        ex = H @ v.astype(np.float64)
+        bound = 2 * math.log2(D) * 2.0 ** -24 * np.sum(np.abs(v.astype(np.float64)))
+        assert np.max(np.abs(O.fwht_f32(v) - ex)) <= bound, D
+
+
+def check_kv4_quant_example():
+    for kind, a in load_kv_example():
+        if kind != "quant":
+            continue
+        vals = [float(v) for v in a["y"].split(",")]
+        y = np.zeros(32, dtype=np.float32)
+        y[:len(vals)] = vals
+        code, sb = O.kv4_quantize_block(y)
+        want = [int(c) for c in a["codes"].split(",")]
+        assert sb == int(a["scale"], 16), f"scale {sb:#x}"
+        assert list(code[:len(want)]) == want and np.all(code[len(want):] == int(a["rest"])), code
+
+
+def check_kv4_encode_examples():
+    for kind, a in load_kv_example():
+        if kind != "enc":
+            continue
+        D = int(a["D"])
+        H = hadamard(D)
+        what, arg = a["x"].split(":")
+        xv = np.zeros(D) if what == "onehot" else H[:, int(arg)].copy()
+        if what == "onehot":
+            xv[int(arg)] = 1.0
+        codes, scales = O.kv4_encode(bf16_bits(xv)[None, :])
+        want = np.full(D // 2, int(a["byte"], 16), dtype=np.uint8)
+        if "byte_at" in a:
+            i, b = a["byte_at"].split(":")
+            want[int(i)] = int(b, 16)
+        assert np.array_equal(codes[0], want), codes
+        assert [int(v) for v in scales[0]] == [int(v, 16) for v in a["scales"].split(",")], scales
+        out, bits = O.kv4_decode(codes, scales)
+        if "at" in a:
+            i, v = a["at"].split(":")
+            exp = np.zeros(D)
+            exp[int(i)] = float(v)
+            assert np.allclose(out[0], exp, rtol=1e-14, atol=1e-15), out[0][:4]
+            bi, bv = a["bf16_at"].split(":")
+            assert int(bits[0, int(bi)]) == int(bv, 16) and int(np.count_nonzero(bits[0])) == 1
+        else:
+            col = H[:, int(a["sign"].split(":")[1])]
+            assert np.allclose(out[0], col * float(a["abs"]), rtol=1e-14, atol=0)
+            bf = int(a["bf16_abs"], 16)
+            assert np.array_equal(bits[0], np.where(col > 0, bf, bf | 0x8000).astype(np.uint16))
+
+
+def _exact_rotation(x_bits):
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    D = x.shape[1]
+    return x, x @ hadamard(D).T / math.sqrt(D)
+
+
+def _nibbles(codes):
+    D = codes.shape[1] * 2
+    c = np.empty((codes.shape[0], D), dtype=np.int64)
+    c[:, 0::2] = codes & 15
+    c[:, 1::2] = codes >> 4
+    return c
+
+
+def check_kv4_codes_match_exact_rounding():
+    for D, seed in ((64, 21), (128, 22), (256, 23)):
+        xb = kv_rows(seed, 96, D)
+        codes, scales = O.kv4_encode(xb)
+        _, y = _exact_rotation(xb)
+        s = scales.view(np.float16).astype(np.float64)
+        yb = y.reshape(y.shape[0], D // 32, 32)
+        t = np.abs(yb).max(axis=2) / 7.0
+        want_s = np.array([[fp16_rne_exact(float(v)) for v in row] for row in t], dtype=np.uint16)
+        # the fp32 rotation may move t across an fp16 midpoint only when t sits
+        # within its error bound of one
+        frac = t / 2.0 ** (np.floor(np.log2(t)) - 10)
+        near_mid = np.abs(frac - np.floor(frac) - 0.5) < 1e-4
+        assert np.all((scales == want_s) | near_mid), "block scales differ from fp16(absmax / 7)"
+        q = np.clip(np.rint(yb / s[:, :, None]), -7, 7).reshape(y.shape)
+        ratio = (yb / s[:, :, None]).reshape(y.shape)
+        tie = np.abs(np.abs(ratio - np.floor(ratio)) - 0.5) < 1e-4
+        ok = (_nibbles(codes) - 8 == q) | tie
+        assert np.all(ok) and np.mean(tie) < 0.01, "codes differ from round(y / s)"
+
+
+def check_kv4_roundtrip_bound():
+    for D, seed in ((64, 31), (128, 32), (256, 33)):
+        xb = kv_rows(seed, 64, D)
+        codes, scales = O.kv4_encode(xb)
+        x, y = _exact_rotation(xb)
+        out, bits = O.kv4_decode(codes, scales)
+        s = np.repeat(scales.view(np.float16).astype(np.float64), 32, axis=1)
+        yq = (_nibbles(codes) - 8) * s
+        # per element in the rotated domain: within half a step (plus the fp32
+        # rotation's own error)
+        assert np.all(np.abs(y - yq) <= s / 2 + 1e-5 * np.abs(y).max(axis=1, keepdims=True)), D
+        # the decode is the orthonormal inverse: equal 2-norm of the error
+        e_rot = np.linalg.norm(y - yq, axis=1)
+        e_x = np.linalg.norm(x - out, axis=1)
+        assert np.allclose(e_x, e_rot, rtol=1e-9, atol=1e-12), D
+        dec = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        assert np.all(np.abs(dec - out) <= np.abs(out) * 2.0 ** -8 + 1e-38), D
+
+
+def check_kv4_single_code_decode():
+    for D in (64, 128, 256):
+        H = hadamard(D)
+        for i in (0, 7, D // 2 + 5, D - 1):
+            c = np.full(D, 8, dtype=np.uint8)
+            c[i] = 9 if i % 3 else 6  # q = +1 or -2
+            codes = (c[0::2] | (c[1::2] << 4)).astype(np.uint8)[None, :]
+            scales = np.full((1, D // 32), 0x3800, dtype=np.uint16)  # 0.5
+            out, _ = O.kv4_decode(codes, scales)
+            want = H[:, i] * (int(c[i]) - 8) * 0.5 / math.sqrt(D)
+            assert np.allclose(out[0], want, rtol=1e-15, atol=0), (D, i)
+
+
+def check_kv4_zero_and_saturation():
+    for D in (64, 256):
+        codes, scales = O.kv4_encode(np.zeros((1, D), dtype=np.uint16))
+        assert np.all(codes == 0x88) and np.all(scales == 0)
+        out, bits = O.kv4_decode(codes, scales)
+        assert np.all(out == 0) and np.all(bits == 0)
+    # constant row of 61952 (a bf16 value): y = 61952 * sqrt(64) e_0 = 495616,
+    # absmax / 7 above the largest half -> s saturates at 65504 (0x7bff);
+    # 495616 / 65504 = 7.57 rounds to 8 and is clamped to 7 (code 15)
+    codes, scales = O.kv4_encode(bf16_bits(np.full((1, 64), 61952.0)))
+    assert int(scales[0, 0]) == 0x7BFF and int(scales[0, 1]) == 0, scales
+    want = np.full(32, 0x88, dtype=np.uint8)
+    want[0] = 0x8F
+    assert np.array_equal(codes[0], want), codes
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

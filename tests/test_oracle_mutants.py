@@ -40,6 +40,24 @@ MUTANTS = [
     ("bf16_truncate", "double r = nearbyint(v / q) * q;", "double r = trunc(v / q) * q;"),
     ("fp16_subnormal", "v = ldexp((double)mant, -24);", "v = ldexp((double)mant, -25);"),
     ("residual_in_double", "x[i] = (float)((double)x[i] + y[i]);", "x[i] = (float)((double)x[i] + (float)y[i] * 1.0000001);"),
+    ("kv_fwht_sign", "v[i + h] = a - b;", "v[i + h] = b - a;"),
+    ("kv_fwht_last_stage", "for (int h = 1; h < D; h *= 2)", "for (int h = 1; h < D / 2; h *= 2)"),
+    ("kv_norm_dropped", "y[i] = y[i] * r;", "y[i] = y[i];"),
+    ("kv_scale_over_8", "float t = amax / 7.0f;", "float t = amax / 8.0f;"),
+    ("kv_round_half_away", "float r = rintf(y[i] / s);", "float r = roundf(y[i] / s);"),
+    ("kv_clamp_8", "q = r > 7.0f ? 7 :", "q = r > 7.0f ? 8 :"),
+    ("kv_no_saturation", "if (t > 65504.0f)\n        t = 65504.0f;", "if (t > 65504.0f)\n        t = t;"),
+    ("kv_code_offset", "code[i] = (uint8_t)(q + 8);", "code[i] = (uint8_t)(q + 7);"),
+    ("kv_nibble_order", "(uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));", "(uint8_t)(q[2 * j + 1] | (q[2 * j] << 4));"),
+    ("kv_dec_sign", "acc += oracle_hadamard_sign(j, i) * y[i];", "acc += oracle_hadamard_sign(j, i ^ 1) * y[i];"),
+    ("kv_dec_nibble", ">> (4 * (i % 2))) & 15;", ">> (4 * (1 - i % 2))) & 15;"),
+    ("kv_dec_scale_block", "oracle_fp16_to_double(scales[(size_t)row * (D / 32) + i / 32]);",
+     "oracle_fp16_to_double(scales[(size_t)row * (D / 32) + i / 64]);"),
+    ("kv_dec_offset", "y[i] = (c - 8) *", "y[i] = (c - 7.5) *"),
+    ("kv_dec_norm", "out[(size_t)row * D + j] = acc * inv;", "out[(size_t)row * D + j] = acc / D;"),
+    ("hadamard_parity", "p ^= (int)(m & 1u);", "p ^= (int)((m >> 1) & 1u);"),
+    ("fp16_subnormal_quantum", "qe = -24; /* subnormal range", "qe = -25; /* subnormal range"),
+    ("fp16_no_carry", "n /= 2.0;\n        qe += 1;", "n -= 1.0;"),
     ("combine_weight_dropped", "y[(size_t)t * d + i] += w[(size_t)t * k + j] * o[i];", "y[(size_t)t * d + i] += o[i];"),
 ]
 
