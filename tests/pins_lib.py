@@ -632,6 +632,12 @@ def check_kv4_zero_and_saturation():
         assert np.all(codes == 0x88) and np.all(scales == 0)
         out, bits = O.kv4_decode(codes, scales)
         assert np.all(out == 0) and np.all(bits == 0)
+    # a row too small for any half scale: x = 1e-8 e_0 gives y = 1.25e-9
+    # everywhere, absmax / 7 underflows fp16 to zero -> every code 8
+    x = np.zeros((1, 64))
+    x[0, 0] = 1e-8
+    codes, scales = O.kv4_encode(bf16_bits(x))
+    assert np.all(scales == 0) and np.all(codes == 0x88), codes
     # constant row of 61952 (a bf16 value): y = 61952 * sqrt(64) e_0 = 495616,
     # absmax / 7 above the largest half -> s saturates at 65504 (0x7bff);
     # 495616 / 65504 = 7.57 rounds to 8 and is clamped to 7 (code 15)
