@@ -685,6 +685,173 @@ def cpu_baseline(w, seconds):
                       + (f" x{w.layers} layers" if w.layers > 1 else "")}
 
 
+# ---------------------------------------------------------------- KV codec
+
+
+KV_STEPS = 50
+KV_KERNELS = ("k_kv4_encode<128>", "k_kv4_decode<128>")
+
+
+def kv_bytes(w) -> int:
+    """Algorithmic bytes of one encode (or one decode) launch over all rows:
+    bf16 rows (2 bytes per value) + codes (0.5) + fp16 scales (1/16)."""
+    return w.rows * w.D * 2 + w.rows * w.D // 2 + w.rows * (w.D // 32) * 2
+
+
+def kv_cpu_baseline(w, seconds):
+    """The oracle's encode + decode on the host, on consecutive rows of the
+    same workload until the time budget is spent."""
+    import oracle
+    import synth
+    oracle.load()
+    el = 0.0  # oracle time only; drawing the rows is not timed
+    rows = 0
+    chunk = 2048
+    while el < seconds or rows == 0:
+        x = synth.gen_kv_rows(w.seed, chunk, w.D, row0=rows)
+        t1 = time.perf_counter()
+        c, sc = oracle.kv4_encode(x)
+        oracle.kv4_decode(c, sc)
+        el += time.perf_counter() - t1
+        rows += chunk
+    return {"value": rows / (w.kv_heads * 2) / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} rows ({rows // (w.kv_heads * 2)} tokens) of {w.name}, encode + fp64 decode"}
+
+
+def measure_kv(S, w, args, world, rank, local):
+    """The codec over one layer's 128K-token K and V cache: a step encodes every
+    row and decodes every row; encode writes one of two code buffers while
+    decode reads the other (written a step earlier, since evicted from L2)."""
+    import torch
+    import synth.device as sdev
+    hbm, _, _, peak_src = load_peaks()
+    steps = args.steps if args.steps is not None else KV_STEPS
+    n, D = w.rows, w.D
+    dev = torch.device("cuda", local)
+    x = sdev.kv_rows(w.seed, n, D)
+    codes = [torch.empty((n, D // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
+    scales = [torch.empty((n, D // 32), dtype=torch.int16, device=dev) for _ in range(2)]
+    out = torch.empty((n, D), dtype=torch.bfloat16, device=dev)
+    S.strata_kv4_encode(x, n, D, codes[1], scales[1])
+    st = torch.cuda.current_stream()
+
+    def step(i):
+        a, b = i % 2, (i + 1) % 2
+        S.strata_kv4_encode(x, n, D, codes[a], scales[a])
+        S.strata_kv4_decode(codes[b], scales[b], n, D, out)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(st)
+    for i in range(steps):
+        e0, e1, e2 = ev[i]
+        e0.record(st)
+        S.strata_kv4_encode(x, n, D, codes[i % 2], scales[i % 2])
+        e1.record(st)
+        S.strata_kv4_decode(codes[(i + 1) % 2], scales[(i + 1) % 2], n, D, out)
+        e2.record(st)
+    t_end.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = dist_max(t_start.elapsed_time(t_end), world)
+    enc_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    ms_step = ms / steps
+    value = w.tokens * steps * world / (ms / 1e3)
+    print(f"# {w.name}: {ms_step * 1e3:.2f} us/step (encode {enc_ms * 1e3:.2f} us, decode {dec_ms * 1e3:.2f} us), "
+          f"{value:.4g} tokens/s", file=sys.stderr, flush=True)
+    nb = kv_bytes(w)
+    kern = {"encode": {"avg_launch_ms": enc_ms, "achieved_gbs": nb / (enc_ms * 1e-3) / 1e9,
+                       "frac": nb / (enc_ms * 1e-3) / 1e9 / hbm},
+            "decode": {"avg_launch_ms": dec_ms, "achieved_gbs": nb / (dec_ms * 1e-3) / 1e9,
+                       "frac": nb / (dec_ms * 1e-3) / 1e9 / hbm}}
+    dom = "encode" if enc_ms >= dec_ms else "decode"
+    dms = kern[dom]["avg_launch_ms"]
+    ach = nb / (dms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": KV_KERNELS[0 if dom == "encode" else 1], "achieved": ach, "peak": hbm,
+            "unit": "GB/s", "frac": ach / hbm, "traffic": None, "traffic_note": "no capture of this shape",
+            "algorithmic_bytes_per_launch": nb,
+            "bytes_basis": "bf16 rows + 4-bit codes + fp16 scales, each moved once",
+            "avg_launch_ms": dms, "avg_launch_ms_source": "CUDA events around each launch on its stream",
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "kernels": kern}
+    e2e = kv_end_to_end(S, w, x, codes[0], scales[0], out, min(steps, 8), world)
+    block = {
+        "metric": "4-bit rotated KV codec: cached tokens/s (one layer's K and V encoded + decoded)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (bf16 rows in and out, 4-bit codes + fp16 scales)",
+        "data": "synthetic (seeded N(0,1) rows, 4 outlier channels x16)",
+        "config": {"workload": w.name, "tokens": w.tokens, "kv_heads": w.kv_heads, "head_dim": D, "rows": n,
+                   "l2": (f"inputs larger than L2 ({nb / 1e9:.2f} GB per launch); decode reads the codes the "
+                          "previous step wrote"),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": roof, "clocks": clk, "e2e": e2e, "gpu_launches": 2 * steps,
+    }
+    del x, codes, scales, out
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        block["cpu_baseline"] = kv_cpu_baseline(w, args.cpu_seconds)
+    return block
+
+
+def kv_end_to_end(S, w, x, codes, scales, out, steps, world):
+    """Through the C ABI from pinned host rows to pinned host rows: per step
+    the rows go up, are encoded and decoded, and the decoded rows come back."""
+    import torch
+    n, D = w.rows, w.D
+    hx = torch.empty((n, D), dtype=torch.bfloat16, pin_memory=True)
+    hx.copy_(x, non_blocking=False)
+    ho = torch.empty((n, D), dtype=torch.bfloat16, pin_memory=True)
+    st = torch.cuda.current_stream()
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        x.copy_(hx, non_blocking=True)
+        S.strata_kv4_encode(x, n, D, codes, scales)
+        S.strata_kv4_decode(codes, scales, n, D, out)
+        ho.copy_(out, non_blocking=True)
+    b.record(st)
+    torch.cuda.synchronize()
+    ms = dist_max(a.elapsed_time(b), world)
+    nbytes = n * D * 2
+    return {"value": w.tokens * steps * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": nbytes, "steps": steps}
+
+
+def kv_reference_block(w, args, world):
+    steps = args.steps if args.steps is not None else 3
+    budget = args.cpu_seconds / max(1, steps + args.warmup)
+    vals = []
+    b = None
+    for i in range(args.warmup + steps):
+        b = kv_cpu_baseline(w, budget)
+        if i >= args.warmup:
+            vals.append(b["value"])
+    value = float(np.mean(vals))
+    return {"metric": "4-bit rotated KV codec: cached tokens/s (one layer's K and V encoded + decoded)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * w.tokens / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 encode, f64 decode", "data": "synthetic (seeded)",
+            "impl": "reference", "config": {"workload": w.name, "tokens": w.tokens, "kv_heads": w.kv_heads,
+                                            "head_dim": w.D, "rows": w.rows},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {b['sample']}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def workloads_of(args):
     """(top-level workload, nested blocks): the default run is the one-token
     decode layer with the 8,192-token prefill layer nested."""
@@ -719,6 +886,10 @@ def run_reference(args, world, rank):
     """The oracle timed on the host cores on this arm's workloads (rank 0 only)."""
     if rank != 0:
         return
+    import synth
+    if args.workload in synth.KV_WORKLOADS:
+        print(json.dumps(kv_reference_block(synth.KV_WORKLOADS[args.workload], args, world)), flush=True)
+        return
     top, nested = workloads_of(args)
     out = reference_block(top, args, world)
     for key, w in nested:
@@ -731,6 +902,12 @@ def run_reference(args, world, rank):
 
 def run_strata(args, world, rank, local):
     import bit_quantized_moe_warp_b200 as S
+    import synth
+    if args.workload in synth.KV_WORKLOADS:
+        out = measure_kv(S, synth.KV_WORKLOADS[args.workload], args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        return
     top, nested = workloads_of(args)
     out = measure(S, top, args, world, rank, local)
     for key, w in nested:
@@ -744,8 +921,9 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=None, choices=list(DEFAULT_STEPS),
-                    help="one workload only (default: decode, with the prefill layer nested)")
+    ap.add_argument("--workload", default=None, choices=list(DEFAULT_STEPS) + ["kv4_128k"],
+                    help="one workload only (default: decode, with the prefill layer nested); kv4_128k: "
+                         "the 4-bit rotated KV-cache codec")
     ap.add_argument("--impl", default="strata", choices=["strata", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

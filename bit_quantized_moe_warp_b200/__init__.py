@@ -40,6 +40,7 @@ STRATA_FORCE_PREFILL = 2
 STRATA_DECODE_MAX_TOKENS = 16
 STRATA_Q2_TILE_BYTES = 1280
 STRATA_Q4_TILE_BYTES = 2304
+STRATA_KV4_BLOCK = 32  # include/strata_kv.h
 FORMAT_OF_BITS = {2: STRATA_FMT_Q2_0_TILED, 4: STRATA_FMT_Q4_0_TILED}
 
 
@@ -82,6 +83,10 @@ _SIGS = {
     "strata_selftest_wait_timeout": (I32, [ctypes.c_uint64, V]),
     "strata_selftest_bounds_check": (I32, [V]),
     "strata_is_checked_build": (I32, []),
+    "strata_kv4_code_bytes": (SZ, [ctypes.c_int64, I32]),
+    "strata_kv4_scale_bytes": (SZ, [ctypes.c_int64, I32]),
+    "strata_kv4_encode": (I32, [V, ctypes.c_int64, I32, V, V, V]),
+    "strata_kv4_decode": (I32, [V, V, ctypes.c_int64, I32, V, V]),
     "strata_status_string": (ctypes.c_char_p, [I32]),
     "strata_last_error": (ctypes.c_char_p, []),
 }
@@ -193,6 +198,24 @@ def strata_moe_stack_forward(layer, router_w, router_bias, expert_blobs, x_resid
     _check(_lib.strata_moe_stack_forward(layer, n, ctypes.cast(W, V), None if B is None else ctypes.cast(B, V),
                                          ctypes.cast(X, V), _ptr(x_resid), n_tokens, float(rms_eps),
                                          _stream(stream)))
+
+
+def strata_kv4_code_bytes(n_rows, head_dim):
+    return _lib.strata_kv4_code_bytes(n_rows, head_dim)
+
+
+def strata_kv4_scale_bytes(n_rows, head_dim):
+    return _lib.strata_kv4_scale_bytes(n_rows, head_dim)
+
+
+def strata_kv4_encode(x, n_rows, head_dim, codes, scales, stream=None):
+    """bf16 rows [n_rows, head_dim] -> 4-bit codes [n_rows, head_dim/2] and fp16 scales [n_rows, head_dim/32]."""
+    _check(_lib.strata_kv4_encode(_ptr(x), n_rows, head_dim, _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def strata_kv4_decode(codes, scales, n_rows, head_dim, out, stream=None):
+    """4-bit codes and fp16 scales of n_rows rows -> bf16 rows [n_rows, head_dim]."""
+    _check(_lib.strata_kv4_decode(_ptr(codes), _ptr(scales), n_rows, head_dim, _ptr(out), _stream(stream)))
 
 
 def strata_rmsnorm_bf16(x, out, n_tokens, d, eps, stream=None):

@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libstrata_moe.so")
 # the same sources with every data-derived index bounds-checked into the status word
 OUT_CHECKED = os.path.join(HERE, "libstrata_moe_checked.so")
-SOURCES = ["strata_moe.cu", "route.cu", "decode_fused.cu", "prefill_gemm.cu", "misc.cu", "route_noalloc.cu", "router_gemm.cu"]
+SOURCES = ["strata_moe.cu", "route.cu", "decode_fused.cu", "prefill_gemm.cu", "misc.cu", "route_noalloc.cu", "router_gemm.cu", "kv_codec.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
@@ -21,7 +21,8 @@ def needs_build(out: str = OUT) -> bool:
         return True
     t = os.path.getmtime(out)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
-    deps.append(os.path.join(HERE, "..", "include", "strata_moe.h"))
+    inc = os.path.join(HERE, "..", "include")
+    deps += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 

@@ -54,6 +54,8 @@ TAG_ROUTER_W = 2
 TAG_CODES = 3
 TAG_SCALES = 4
 TAG_PERM = 5
+TAG_KV = 6
+TAG_KV_OUTLIERS = 7
 
 # matrix ids inside one expert
 GATE, UP, DOWN = 0, 1, 2
@@ -245,6 +247,59 @@ WORKLOADS = {
     "verify4_q4": Workload("verify4_q4", 2048, 768, 512, 10, 4, 1, True, 6, bits=4),
     "prefill_q4": Workload("prefill_q4", 2048, 768, 512, 10, 8192, 1, True, 6, bits=4),
 }
+
+
+# ----------------------------------------------------------------------------
+# KV-cache rows for the 4-bit rotated codec
+
+
+@dataclasses.dataclass(frozen=True)
+class KvWorkload:
+    """One attention layer's K and V cache: tokens x kv_heads x 2 rows of D."""
+    name: str
+    tokens: int
+    kv_heads: int
+    D: int
+    seed: int
+
+    @property
+    def rows(self) -> int:
+        return self.tokens * self.kv_heads * 2
+
+    def desc(self) -> str:
+        return (f"tokens={self.tokens} kv_heads={self.kv_heads} head_dim={self.D} rows={self.rows} "
+                f"outlier_channels=4x16 seed={self.seed}")
+
+
+# a 128K-token context ("Strata：把 125B 大模型塞进 12GB 显卡…", 长上下文: the 4-bit
+# cache is quoted at 128K); head_dim 128 and 4 KV heads are assumed shapes
+KV_WORKLOADS = {
+    "kv4_128k": KvWorkload("kv4_128k", 131072, 4, 128, 7),
+}
+
+KV_OUTLIERS = 4  # channels per head_dim scaled by 16 (an exact power of two)
+
+
+def kv_outlier_channels(seed: int, D: int) -> np.ndarray:
+    """The fixed channels (same in every row) that carry outliers."""
+    w = words(stream_key(seed, TAG_KV_OUTLIERS), 0, 64)
+    out = []
+    for v in w:
+        c = int(v % np.uint64(D))
+        if c not in out:
+            out.append(c)
+        if len(out) == KV_OUTLIERS:
+            break
+    return np.array(sorted(out), dtype=np.int64)
+
+
+def gen_kv_rows(seed: int, rows: int, D: int, row0: int = 0) -> np.ndarray:
+    """Cached key/value rows, uint16 bf16 bits [rows, D]: bf16(z), z ~ N(0,1),
+    times 16 in the outlier channels (exact in bf16), rows row0.."""
+    z = f32_to_bf16_bits(normals(stream_key(seed, TAG_KV), rows * D, start=row0 * D)).reshape(rows, D)
+    ch = kv_outlier_channels(seed, D)
+    z[:, ch] = f32_to_bf16_bits(bf16_bits_to_f32(z[:, ch]) * np.float32(16.0))
+    return z
 
 
 def router_bias(w: Workload, layer: int):

@@ -9,8 +9,8 @@ import subprocess
 
 import numpy as np
 
-from . import (DOWN, GATE, TAG_CODES, TAG_ROUTER_W, TAG_SCALES, TAG_X, UP, Workload, router_bias,
-               stream_key)
+from . import (DOWN, GATE, TAG_CODES, TAG_KV, TAG_ROUTER_W, TAG_SCALES, TAG_X, UP, Workload, kv_outlier_channels,
+               router_bias, stream_key)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "synth_dev.cu")
@@ -58,6 +58,16 @@ def x_bf16(seed: int, T: int, d: int, stream: int = 0, tok0: int = 0):
     import torch
     out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
     _chk(_load().synth_x_bf16(stream_key(seed, TAG_X, stream), tok0 * d, T * d, out.data_ptr(), _stream()))
+    return out
+
+
+def kv_rows(seed: int, rows: int, D: int, row0: int = 0):
+    """torch.bfloat16 [rows, D] on the current device (same as synth.gen_kv_rows)."""
+    import torch
+    out = torch.empty((rows, D), dtype=torch.bfloat16, device="cuda")
+    _chk(_load().synth_x_bf16(stream_key(seed, TAG_KV), row0 * D, rows * D, out.data_ptr(), _stream()))
+    ch = torch.from_numpy(kv_outlier_channels(seed, D)).cuda()
+    out[:, ch] *= 16  # exact in bf16
     return out
 
 

@@ -463,14 +463,8 @@ def bf16_bits(v) -> np.ndarray:
 
 
 def kv_rows(seed: int, rows: int, D: int) -> np.ndarray:
-    """bf16 rows, N(0,1) with a few large outliers per row (cached keys and
-    values carry such channels)."""
-    rng = np.random.default_rng(seed)
-    x = rng.standard_normal((rows, D)).astype(np.float32)
-    big = rng.integers(0, D, (rows, 2))
-    for r in range(rows):
-        x[r, big[r]] *= 20.0
-    return bf16_bits(x)
+    """bf16 cache rows from the seeded generator: N(0,1) with outlier channels."""
+    return synth.gen_kv_rows(seed, rows, D)
 
 
 def load_kv_example():

@@ -14,7 +14,7 @@ import pins_lib
 import synth
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "strata_moe.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -28,7 +28,7 @@ def S():
 
 
 def header_functions():
-    src = open(HEADER).read()
+    src = "".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(strata_[a-z0-9_]+)\s*\(", src)))
 
@@ -159,12 +159,12 @@ def test_status_strings(S):
 
 def test_binding_constants_match_header(S):
     """Every #define the binding restates has the header's value."""
-    src = open(HEADER).read()
+    src = "".join(open(h).read() for h in HEADERS)
     defs = dict(re.findall(r"#define\s+(STRATA_[A-Z0-9_]+)\s+\(?([0-9]+)u?\b", src))
     restated = [n for n in dir(S) if n.startswith("STRATA_") and n in defs]
     assert {"STRATA_Q2_TILE_BYTES", "STRATA_ACCUMULATE", "STRATA_FORCE_PREFILL",
             "STRATA_DECODE_MAX_TOKENS", "STRATA_FMT_Q2_0_TILED", "STRATA_FMT_Q4_0_TILED",
-            "STRATA_Q4_TILE_BYTES"} <= set(restated)
+            "STRATA_Q4_TILE_BYTES", "STRATA_KV4_BLOCK"} <= set(restated)
     for n in restated:
         assert getattr(S, n) == int(defs[n]), n
 
@@ -181,3 +181,36 @@ def test_checked_build_exports_the_same_calls(S):
     lib.strata_is_checked_build.restype = ctypes.c_int32
     assert lib.strata_is_checked_build() == 1
     assert S.strata_is_checked_build() == 0
+
+
+def test_kv4_sizes_and_refusals(S):
+    """Sizes of the 4-bit KV format and the codec's argument checks, all of
+    which return before any device work (no GPU needed)."""
+    assert S.strata_kv4_code_bytes(1000, 128) == 64000
+    assert S.strata_kv4_scale_bytes(1000, 128) == 8000
+    assert S.strata_kv4_code_bytes(3, 256) == 384 and S.strata_kv4_scale_bytes(3, 64) == 12
+    assert S.strata_kv4_code_bytes(10, 96) == 0 and S.strata_kv4_scale_bytes(-1, 128) == 0
+    for D in (32, 96, 512, 0):
+        with pytest.raises(S.StrataError) as e:
+            S.strata_kv4_encode(0x1000, 4, D, 0x2000, 0x3000, stream=0)
+        assert e.value.status == S.STRATA_ERR_UNSUPPORTED
+        with pytest.raises(S.StrataError) as e:
+            S.strata_kv4_decode(0x2000, 0x3000, 4, D, 0x1000, stream=0)
+        assert e.value.status == S.STRATA_ERR_UNSUPPORTED
+    bad = [dict(x=0x1000, n=-1, c=0x2000, s=0x3000),  # negative row count
+           dict(x=0, n=4, c=0x2000, s=0x3000),  # NULL input
+           dict(x=0x1000, n=4, c=0, s=0x3000),
+           dict(x=0x1000, n=4, c=0x2000, s=0),
+           dict(x=0x1008, n=4, c=0x2000, s=0x3000),  # x not 16-byte aligned
+           dict(x=0x1000, n=4, c=0x2002, s=0x3000),  # codes not 4-byte aligned
+           dict(x=0x1000, n=4, c=0x2000, s=0x3001)]  # scales not 2-byte aligned
+    for a in bad:
+        with pytest.raises(S.StrataError) as e:
+            S.strata_kv4_encode(a["x"], a["n"], 128, a["c"], a["s"], stream=0)
+        assert e.value.status == S.STRATA_ERR_INVALID_ARG, a
+        with pytest.raises(S.StrataError) as e:
+            S.strata_kv4_decode(a["c"], a["s"], a["n"], 128, a["x"], stream=0)
+        assert e.value.status == S.STRATA_ERR_INVALID_ARG, a
+    # zero rows: nothing to do, even with NULL buffers
+    S.strata_kv4_encode(0, 0, 128, 0, 0, stream=0)
+    S.strata_kv4_decode(0, 0, 0, 128, 0, stream=0)
