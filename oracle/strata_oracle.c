@@ -46,7 +46,8 @@
  *    row (D a power of two, H the Sylvester matrix, H[i][j] =
  *    (-1)^popcount(i & j)); 32-value blocks with one fp16 scale
  *    s = fp16(absmax / 7) (saturated at 65504); q = round-half-even of
- *    y * fp32(1 / s), clamped to [-7, 7], stored as the nibble q + 8;
+ *    the exact product y * fp32(1 / s), clamped to [-7, 7], stored as the
+ *    nibble q + 8;
  *    decoding inverts:
  *    x = H ((c - 8) s) / sqrt(D), rounded to bf16. Because the codes are
  *    integers decided by floating point, the encoder computes in fp32 in a
@@ -427,10 +428,11 @@ void oracle_fwht_f32(int D, float *v)
 }
 
 /* One 32-value block: s = fp16(min(absmax / 7, 65504)), all in fp32;
- * q_i = clamp(rint(y_i * fp32(1 / s)), -7, 7) (q = 0 when s is zero);
- * code q_i + 8. The quotient is taken through the fp32 reciprocal of s (the
- * precision the GPU decides in); it differs from an exactly rounded y / s
- * only within a few fp32 ulps of a half-integer. */
+ * q_i = clamp(rint(y_i * fp32(1 / s)), -7, 7) (q = 0 when s is zero), the
+ * product taken exactly and rounded once, to the nearest integer, ties to
+ * even; code q_i + 8. The quotient goes through the fp32 reciprocal of s
+ * (the precision the GPU decides in); it differs from an exactly rounded
+ * y / s only within a few fp32 ulps of a half-integer. */
 void oracle_kv4_quantize_block(const float *y, uint8_t *code, uint16_t *scale_bits)
 {
     float amax = 0.0f;
@@ -444,8 +446,8 @@ void oracle_kv4_quantize_block(const float *y, uint8_t *code, uint16_t *scale_bi
     float s = (float)oracle_fp16_to_double(sb);
     float inv = s > 0.0f ? 1.0f / s : 0.0f;
     for (int i = 0; i < 32; ++i) {
-        float r = rintf(y[i] * inv); /* default rounding mode: ties to even */
-        int q = r > 7.0f ? 7 : (r < -7.0f ? -7 : (int)r);
+        double r = rint((double)y[i] * (double)inv); /* exact product; ties to even */
+        int q = r > 7.0 ? 7 : (r < -7.0 ? -7 : (int)r);
         code[i] = (uint8_t)(q + 8);
     }
     *scale_bits = sb;

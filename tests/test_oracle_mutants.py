@@ -44,8 +44,9 @@ MUTANTS = [
     ("kv_fwht_last_stage", "for (int h = 1; h < D; h *= 2)", "for (int h = 1; h < D / 2; h *= 2)"),
     ("kv_norm_dropped", "y[i] = y[i] * r;", "y[i] = y[i];"),
     ("kv_scale_over_8", "float t = amax / 7.0f;", "float t = amax / 8.0f;"),
-    ("kv_round_half_away", "float r = rintf(y[i] * inv);", "float r = roundf(y[i] * inv);"),
-    ("kv_clamp_8", "int q = r > 7.0f ? 7 :", "int q = r > 7.0f ? 8 :"),
+    ("kv_round_half_away", "double r = rint((double)y[i] * (double)inv);", "double r = round((double)y[i] * (double)inv);"),
+    ("kv_product_rounded_first", "double r = rint((double)y[i] * (double)inv);", "double r = rintf(y[i] * inv);"),
+    ("kv_clamp_8", "int q = r > 7.0 ? 7 :", "int q = r > 7.0 ? 8 :"),
     ("kv_zero_scale_inverse", "float inv = s > 0.0f ? 1.0f / s : 0.0f;", "float inv = 1.0f / s;"),
     ("kv_no_saturation", "if (t > 65504.0f)\n        t = 65504.0f;", "if (t > 65504.0f)\n        t = t;"),
     ("kv_code_offset", "code[i] = (uint8_t)(q + 8);", "code[i] = (uint8_t)(q + 7);"),
