@@ -52,6 +52,9 @@ MEASURED_TRAFFIC = {
     "decode_q4": {"bytes": 30853632, "sources": ("decode_fused.cu", "common.cuh", "topk.cuh"), "sha": "e59540585b4c4eee"},
     "prefill": {"bytes": 683609344, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "4c18aa910c077009"},
     "prefill_q4": {"bytes": 872128256, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "4c18aa910c077009"},
+    # dram__bytes.sum.per_second x gpu__time_duration.sum of one launch each
+    "kv4_128k_encode": {"bytes": 316628758, "sources": ("kv_codec.cu",), "sha": "9e6be1d5c333ba3b"},
+    "kv4_128k_decode": {"bytes": 285829414, "sources": ("kv_codec.cu",), "sha": "9e6be1d5c333ba3b"},
 }
 
 # library kernels per single-layer call: decode = the one-launch layer kernel;
@@ -777,8 +780,11 @@ def measure_kv(S, w, args, world, rank, local):
     dom = "encode" if enc_ms >= dec_ms else "decode"
     dms = kern[dom]["avg_launch_ms"]
     ach = nb / (dms * 1e-3) / 1e9
+    traffic, tnote = measured_traffic(f"{w.name}_{dom}")
+    for k in kern:
+        kern[k]["traffic"], _ = measured_traffic(f"{w.name}_{k}")
     roof = {"bound": "hbm", "kernel": KV_KERNELS[0 if dom == "encode" else 1], "achieved": ach, "peak": hbm,
-            "unit": "GB/s", "frac": ach / hbm, "traffic": None, "traffic_note": "no capture of this shape",
+            "unit": "GB/s", "frac": ach / hbm, "traffic": traffic, "traffic_note": tnote,
             "algorithmic_bytes_per_launch": nb,
             "bytes_basis": "bf16 rows + 4-bit codes + fp16 scales, each moved once",
             "avg_launch_ms": dms, "avg_launch_ms_source": "CUDA events around each launch on its stream",

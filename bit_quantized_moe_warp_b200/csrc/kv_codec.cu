@@ -5,17 +5,18 @@
 // bound by HBM bandwidth (encode: 2 + 0.5625 bytes per value, decode the
 // reverse), with the transform's butterflies and the block rule in registers.
 //
-// Value layout in a warp: a row of D values is spread over D/16 consecutive
-// lanes, each holding 16 values as two runs of 8: lane l (of its row) holds
-// values 8 (l + m D/16) + e, m in {0, 1}, e in [0, 8). One 16-byte load per
-// run: a warp instruction reads D/16 x 16 contiguous bytes of each of its
-// rows. Index bits 0..2 (e) and the top bit (m) are inside the lane; the
-// bits in between (l) are crossed with one shuffle per value and stage, so a
-// row needs log2(D/16) shuffle stages (2, 3, 4 for D = 64, 128, 256). The
-// butterfly stages run in the order of their stride, 1, 2, ..., D/2, each
-// pair (a, b) becoming (a + b, a - b) in fp32, which fixes every rounding of
-// the encoder. A 32-value quantisation block is 4 lanes x 8 values: its
-// absmax takes two xor-shuffles.
+// Value layout in a warp: a row of D values is spread over D / (8 R)
+// consecutive lanes (R = 4 runs of 8 values per lane for D >= 128, 2 for
+// D = 64): lane l (of its row) holds values 8 (l + m D / (8 R)) + e for runs
+// m < R and e < 8. One 16-byte load per run: a warp instruction reads
+// D / (8 R) x 16 contiguous bytes of each of its rows. Index bits 0..2 (e)
+// and the top log2(R) bits (m) are inside the lane; the bits in between (l)
+// are crossed with one shuffle per value and stage (2, 2, 3 stages for
+// D = 64, 128, 256). The butterfly stages run in the order of their stride,
+// 1, 2, ..., D/2, each pair (a, b) becoming (a + b, a - b) in fp32, which
+// fixes every rounding of the encoder; from stride 2 on, two butterflies go
+// through one packed fp32x2 instruction. A 32-value quantisation block is 4
+// lanes x 8 values: its absmax takes two xor-shuffles.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -27,15 +28,19 @@
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 2;  // row groups whose loads a warp issues before computing
 constexpr unsigned kFull = 0xffffffffu;
+// 1.5 * 2^23 + 8: added to p with |p| < 2^22 it leaves rint(p) + 8 (ties to
+// even) in the low mantissa bits
+constexpr float kRound8 = 12582920.f;
 
 template <int D>
 struct KvRow {
-    static constexpr int kLanes = D / 16;              // lanes per row
-    static constexpr int kRowsPerWarp = 32 / kLanes;   // rows per warp instruction
-    static constexpr int kVec = D / 8;                 // 16-byte chunks of bf16 (and 4-byte code words) per row
-    static constexpr int kBlocks = D / 32;             // scales per row
+    static constexpr int kRuns = D == 64 ? 2 : 4;        // runs of 8 values per lane
+    static constexpr int kLanes = D / (8 * kRuns);       // lanes per row
+    static constexpr int kRowsPerWarp = 32 / kLanes;     // rows per warp instruction
+    static constexpr int kUnroll = 4 / kRuns;            // row groups in flight per warp
+    static constexpr int kVec = D / 8;                   // 16-byte chunks of bf16 (and 4-byte code words) per row
+    static constexpr int kBlocks = D / 32;               // scales per row
 };
 
 // fp32(1 / sqrt(D)), the rotation's normalisation
@@ -48,49 +53,68 @@ __device__ __forceinline__ float inv_sqrt_d<128>() { return 0.088388347648318440
 template <>
 __device__ __forceinline__ float inv_sqrt_d<256>() { return 0.0625f; }
 
-// Unnormalised Walsh-Hadamard transform of the row whose values v[m][e] this
-// lane holds (lane l of the row), stage strides 1, 2, ..., D/2 in order.
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// (a + b, a - b) on two butterflies at once; a - b = fma(-1, b, a) exactly
+__device__ __forceinline__ void bfly2(float2 &a, float2 &b) {
+    const float2 s = __fadd2_rn(a, b);
+    b = __ffma2_rn(f2(-1.f), b, a);
+    a = s;
+}
+
+// Unnormalised Walsh-Hadamard transform of the row whose values this lane
+// holds, x[m][k] = (value 2k, value 2k + 1) of run m; lane l of the row.
 template <int D>
-__device__ __forceinline__ void fwht_row(float (&v)[2][8], int l) {
+__device__ __forceinline__ void fwht_row(float2 (&x)[KvRow<D>::kRuns][4], int l) {
+    using R = KvRow<D>;
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1)
+    for (int m = 0; m < R::kRuns; ++m)
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
+        for (int k = 0; k < 4; ++k) {  // stride 1: the two halves of a pair
+            const float a = x[m][k].x, b = x[m][k].y;
+            x[m][k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+        }
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (!(e & h)) {
-                    const float a = v[m][e], b = v[m][e + h];
-                    v[m][e] = __fadd_rn(a, b);
-                    v[m][e + h] = __fsub_rn(a, b);
-                }
+    for (int m = 0; m < R::kRuns; ++m) {
+        bfly2(x[m][0], x[m][1]);  // stride 2
+        bfly2(x[m][2], x[m][3]);
+        bfly2(x[m][0], x[m][2]);  // stride 4
+        bfly2(x[m][1], x[m][3]);
+    }
 #pragma unroll
-    for (int k = 1; k < KvRow<D>::kLanes; k <<= 1) {
+    for (int k = 1; k < R::kLanes; k <<= 1) {
         // the lane with bit k of l clear holds a, its partner b: the lower lane
         // forms a + b, the upper p - v = a - b (the sign flip is exact)
-        const float sg = (l & k) ? -1.f : 1.f;
+        const float2 sg = f2((l & k) ? -1.f : 1.f);
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
+        for (int m = 0; m < R::kRuns; ++m)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float p = __shfl_xor_sync(kFull, v[m][e], k);
-                v[m][e] = __fmaf_rn(sg, v[m][e], p);
+            for (int j = 0; j < 4; ++j) {
+                const float2 p = make_float2(__shfl_xor_sync(kFull, x[m][j].x, k), __shfl_xor_sync(kFull, x[m][j].y, k));
+                x[m][j] = __ffma2_rn(sg, x[m][j], p);
             }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float a = v[0][e], b = v[1][e];
-        v[0][e] = __fadd_rn(a, b);
-        v[1][e] = __fsub_rn(a, b);
-    }
+    for (int h = 1; h < R::kRuns; h <<= 1)  // the run bits, lowest first
+#pragma unroll
+        for (int m = 0; m < R::kRuns; ++m)
+            if (!(m & h))
+#pragma unroll
+                for (int j = 0; j < 4; ++j) bfly2(x[m][j], x[m + h][j]);
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&v)[8]) {
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float2 (&v)[4]) {
     const uint32_t p[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        v[2 * k] = __uint_as_float(p[k] << 16);
-        v[2 * k + 1] = __uint_as_float(p[k] & 0xffff0000u);
-    }
+    for (int k = 0; k < 4; ++k) v[k] = make_float2(__uint_as_float(p[k] << 16), __uint_as_float(p[k] & 0xffff0000u));
+}
+
+// Codes of one run from the rounded sums z (low nibbles): byte j of the word
+// holds value 2j in its low nibble and 2j + 1 in its high one.
+__device__ __forceinline__ uint32_t pack_nibbles(const uint32_t (&z)[8]) {
+    const uint32_t even = __byte_perm(__byte_perm(z[0], z[2], 0x0040), __byte_perm(z[4], z[6], 0x4000), 0x7610);
+    const uint32_t odd = __byte_perm(__byte_perm(z[1], z[3], 0x0040), __byte_perm(z[5], z[7], 0x4000), 0x7610);
+    return even | (odd << 4);
 }
 
 template <int D>
@@ -102,51 +126,69 @@ __global__ void __launch_bounds__(kThreads) k_kv4_encode(const uint4 *__restrict
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
     const int64_t n_groups = (n_rows + R::kRowsPerWarp - 1) / R::kRowsPerWarp;
     const float r = inv_sqrt_d<D>();
-    for (int64_t g0 = warp * kUnroll; g0 < n_groups; g0 += n_warps * kUnroll) {  // warp-uniform
-        uint4 raw[kUnroll][2];
+    for (int64_t g0 = warp * R::kUnroll; g0 < n_groups; g0 += n_warps * R::kUnroll) {  // warp-uniform
+        uint4 raw[R::kUnroll][R::kRuns];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < R::kUnroll; ++u) {
             const int64_t row = (g0 + u) * R::kRowsPerWarp + rw;
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int m = 0; m < R::kRuns; ++m)
                 raw[u][m] = row < n_rows ? __ldcs(x + row * R::kVec + l + R::kLanes * m) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < R::kUnroll; ++u) {
             const int64_t row = (g0 + u) * R::kRowsPerWarp + rw;
-            float v[2][8];
-            bf16x8_to_f32(raw[u][0], v[0]);
-            bf16x8_to_f32(raw[u][1], v[1]);
-            fwht_row<D>(v, l);
-            uint32_t word[2];
-            uint16_t sbits[2];
+            float2 v[R::kRuns][4];
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
+            for (int m = 0; m < R::kRuns; ++m) bf16x8_to_f32(raw[u][m], v[m]);
+            fwht_row<D>(v, l);
+            uint32_t word[R::kRuns];
+            uint16_t sbits[R::kRuns];
+#pragma unroll
+            for (int m = 0; m < R::kRuns; ++m) {
                 float amax = 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    v[m][e] = __fmul_rn(v[m][e], r);
-                    amax = fmaxf(amax, fabsf(v[m][e]));
+                for (int k = 0; k < 4; ++k) {
+                    v[m][k] = __fmul2_rn(v[m][k], f2(r));
+                    amax = fmaxf(amax, fmaxf(fabsf(v[m][k].x), fabsf(v[m][k].y)));
                 }
                 amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-                const __half hs = __float2half_rn(fminf(__fdiv_rn(amax, 7.f), 65504.f));
+                const float t = __fdiv_rn(amax, 7.f);
+                const __half hs = __float2half_rn(fminf(t, 65504.f));
                 const float s = __half2float(hs);
                 const float inv = s > 0.f ? __frcp_rn(s) : 0.f;
-                uint32_t wd = 0;
+                uint32_t z[8];
+                if (t >= 6.103515625e-05f && t <= 65504.f) {
+                    // s is a normal half within 2^-11 of absmax / 7: |y * inv| < 7.5,
+                    // so one fused multiply-add rounds the exact product, no clamp
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    // clamp, then round half to even by adding 1.5 * 2^23 + 8:
-                    // the sum's low mantissa bits are rint(p) + 8 in [1, 15]
-                    const float p = fminf(fmaxf(__fmul_rn(v[m][e], inv), -7.f), 7.f);
-                    wd |= (__float_as_uint(__fadd_rn(p, 12582920.f)) & 15u) << (4 * e);
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 q = __ffma2_rn(v[m][k], f2(inv), f2(kRound8));
+                        z[2 * k] = __float_as_uint(q.x);
+                        z[2 * k + 1] = __float_as_uint(q.y);
+                    }
+                } else {
+                    // a subnormal or saturated scale: the product may leave [-7.5, 7.5]
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float y = (e & 1) ? v[m][e / 2].y : v[m][e / 2].x;
+                        int q;
+                        if (fabsf(__fmul_rn(y, inv)) >= 8.f) {
+                            q = y > 0.f ? 7 : -7;  // the exact product is beyond 7.5
+                        } else {
+                            q = (int)(__float_as_uint(__fmaf_rn(y, inv, 12582912.f)) - 0x4b400000u);
+                            q = q > 7 ? 7 : (q < -7 ? -7 : q);
+                        }
+                        z[e] = (uint32_t)(q + 8);
+                    }
                 }
-                word[m] = wd;
+                word[m] = pack_nibbles(z);
                 sbits[m] = __half_as_ushort(hs);
             }
             if (row < n_rows) {
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < R::kRuns; ++m) {
                     __stcs(codes + row * R::kVec + l + R::kLanes * m, word[m]);
                     if ((l & 3) == 0) __stcs(scales + row * R::kBlocks + (l + R::kLanes * m) / 4, sbits[m]);
                 }
@@ -165,42 +207,44 @@ __global__ void __launch_bounds__(kThreads) k_kv4_decode(const uint32_t *__restr
     const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
     const int64_t n_groups = (n_rows + R::kRowsPerWarp - 1) / R::kRowsPerWarp;
     const float r = inv_sqrt_d<D>();
-    for (int64_t g0 = warp * kUnroll; g0 < n_groups; g0 += n_warps * kUnroll) {  // warp-uniform
-        uint32_t w[kUnroll][2];
-        uint16_t sb[kUnroll][2];
+    for (int64_t g0 = warp * R::kUnroll; g0 < n_groups; g0 += n_warps * R::kUnroll) {  // warp-uniform
+        uint32_t w[R::kUnroll][R::kRuns];
+        uint16_t sb[R::kUnroll][R::kRuns];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < R::kUnroll; ++u) {
             const int64_t row = (g0 + u) * R::kRowsPerWarp + rw;
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
+            for (int m = 0; m < R::kRuns; ++m) {
                 const bool ok = row < n_rows;
                 w[u][m] = ok ? __ldcs(codes + row * R::kVec + l + R::kLanes * m) : 0x88888888u;
                 sb[u][m] = ok ? __ldcs(scales + row * R::kBlocks + (l + R::kLanes * m) / 4) : (uint16_t)0;
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < R::kUnroll; ++u) {
             const int64_t row = (g0 + u) * R::kRowsPerWarp + rw;
-            float v[2][8];
+            float2 v[R::kRuns][4];
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const float s = __half2float(__ushort_as_half(sb[u][m]));
+            for (int m = 0; m < R::kRuns; ++m) {
+                // (c - 8) * s * fp32(1/sqrt(D)): the normalisation is applied on the
+                // way in (the transform is linear)
+                const float sr = __fmul_rn(__half2float(__ushort_as_half(sb[u][m])), r);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int k = 0; k < 4; ++k) {
                     // 2^23 + c, minus 2^23 + 8: the exact c - 8
-                    const float q = __fsub_rn(__uint_as_float(0x4b000000u | ((w[u][m] >> (4 * e)) & 15u)), 8388616.f);
-                    v[m][e] = __fmul_rn(q, s);
+                    const float2 c = make_float2(__uint_as_float(0x4b000000u | ((w[u][m] >> (8 * k)) & 15u)),
+                                                 __uint_as_float(0x4b000000u | ((w[u][m] >> (8 * k + 4)) & 15u)));
+                    v[m][k] = __fmul2_rn(__fadd2_rn(c, f2(-8388616.f)), f2(sr));
                 }
             }
             fwht_row<D>(v, l);
             if (row < n_rows) {
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < R::kRuns; ++m) {
                     uint32_t o[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const __nv_bfloat162 b2 =
-                            __floats2bfloat162_rn(__fmul_rn(v[m][2 * k], r), __fmul_rn(v[m][2 * k + 1], r));
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[m][k].x, v[m][k].y);
                         o[k] = *reinterpret_cast<const uint32_t *>(&b2);
                     }
                     __stcs(out + row * R::kVec + l + R::kLanes * m, make_uint4(o[0], o[1], o[2], o[3]));
@@ -213,13 +257,13 @@ __global__ void __launch_bounds__(kThreads) k_kv4_decode(const uint32_t *__restr
 // Blocks for n_rows rows: enough warps for every row group, at most the
 // number the device holds at once (a persistent grid-stride loop beyond that).
 template <typename K>
-int grid_for(K kernel, int64_t n_rows, int rows_per_warp, int device) {
+int grid_for(K kernel, int64_t n_rows, int rows_per_warp, int unroll, int device) {
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess || per_sm <= 0)
         per_sm = 1;
     const int64_t groups = (n_rows + rows_per_warp - 1) / rows_per_warp;
-    const int64_t warps = (groups + kUnroll - 1) / kUnroll;
+    const int64_t warps = (groups + unroll - 1) / unroll;
     const int64_t need = (warps + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = (int64_t)sms * per_sm;
     return (int)(need < cap ? need : cap);
@@ -229,7 +273,7 @@ template <int D>
 cudaError_t launch_encode(const void *x, int64_t n, void *codes, void *scales, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
-    const int grid = grid_for(k_kv4_encode<D>, n, KvRow<D>::kRowsPerWarp, dev);
+    const int grid = grid_for(k_kv4_encode<D>, n, KvRow<D>::kRowsPerWarp, KvRow<D>::kUnroll, dev);
     k_kv4_encode<D><<<grid, kThreads, 0, st>>>(static_cast<const uint4 *>(x), n, static_cast<uint32_t *>(codes),
                                               static_cast<uint16_t *>(scales));
     return cudaGetLastError();
@@ -239,7 +283,7 @@ template <int D>
 cudaError_t launch_decode(const void *codes, const void *scales, int64_t n, void *out, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
-    const int grid = grid_for(k_kv4_decode<D>, n, KvRow<D>::kRowsPerWarp, dev);
+    const int grid = grid_for(k_kv4_decode<D>, n, KvRow<D>::kRowsPerWarp, KvRow<D>::kUnroll, dev);
     k_kv4_decode<D><<<grid, kThreads, 0, st>>>(static_cast<const uint32_t *>(codes),
                                               static_cast<const uint16_t *>(scales), n, static_cast<uint4 *>(out));
     return cudaGetLastError();
