@@ -53,8 +53,8 @@ MEASURED_TRAFFIC = {
     "prefill": {"bytes": 683609344, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "4c18aa910c077009"},
     "prefill_q4": {"bytes": 872128256, "sources": ("prefill_gemm.cu", "common.cuh"), "sha": "4c18aa910c077009"},
     # dram__bytes.sum.per_second x gpu__time_duration.sum of one launch each
-    "kv4_128k_encode": {"bytes": 316628758, "sources": ("kv_codec.cu",), "sha": "9e6be1d5c333ba3b"},
-    "kv4_128k_decode": {"bytes": 285829414, "sources": ("kv_codec.cu",), "sha": "9e6be1d5c333ba3b"},
+    "kv4_128k_encode": {"bytes": 316971249, "sources": ("kv_codec.cu",), "sha": "a1739b8effd04803"},
+    "kv4_128k_decode": {"bytes": 286000091, "sources": ("kv_codec.cu",), "sha": "a1739b8effd04803"},
 }
 
 # library kernels per single-layer call: decode = the one-launch layer kernel;

@@ -144,22 +144,57 @@ __global__ void __launch_bounds__(kThreads) k_kv4_encode(const uint4 *__restrict
             fwht_row<D>(v, l);
             uint32_t word[R::kRuns];
             uint16_t sbits[R::kRuns];
+            float amax[R::kRuns];
 #pragma unroll
             for (int m = 0; m < R::kRuns; ++m) {
-                float amax = 0.f;
+                amax[m] = 0.f;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     v[m][k] = __fmul2_rn(v[m][k], f2(r));
-                    amax = fmaxf(amax, fmaxf(fabsf(v[m][k].x), fabsf(v[m][k].y)));
+                    amax[m] = fmaxf(amax[m], fmaxf(fabsf(v[m][k].x), fabsf(v[m][k].y)));
                 }
-                amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-                const float t = __fdiv_rn(amax, 7.f);
-                const __half hs = __float2half_rn(fminf(t, 65504.f));
-                const float s = __half2float(hs);
-                const float inv = s > 0.f ? __frcp_rn(s) : 0.f;
+                amax[m] = fmaxf(amax[m], __shfl_xor_sync(kFull, amax[m], 1));
+                amax[m] = fmaxf(amax[m], __shfl_xor_sync(kFull, amax[m], 2));
+            }
+            // Block scales. With 4 runs a warp holds 8 blocks x 4 runs = 32 (block,
+            // run) pairs, and every lane of a block already has the block's absmax
+            // for each run: lane j computes the scale of run j % 4 of its block once,
+            // and the block's lanes fetch the four results (instead of each lane
+            // computing all four, four times per block).
+            float inv_of[R::kRuns];
+            uint32_t sw_of[R::kRuns];  // scale bits | 1 << 16 when the scale is a normal half
+            {
+                float a = amax[0];
+#pragma unroll
+                for (int m = 1; m < R::kRuns; ++m) a = (lane % R::kRuns) == m ? amax[m] : a;
+                float inv = 0.f;
+                uint32_t sw = 0;
+                if (R::kRuns == 4) {
+                    const float t = __fdiv_rn(a, 7.f);
+                    const __half hs = __float2half_rn(fminf(t, 65504.f));
+                    const float sv = __half2float(hs);
+                    inv = sv > 0.f ? __frcp_rn(sv) : 0.f;
+                    sw = __half_as_ushort(hs) | ((t >= 6.103515625e-05f && t <= 65504.f) ? 0x10000u : 0u);
+                }
+#pragma unroll
+                for (int m = 0; m < R::kRuns; ++m) {
+                    if (R::kRuns == 4) {
+                        inv_of[m] = __shfl_sync(kFull, inv, (lane & ~3) + m);
+                        sw_of[m] = __shfl_sync(kFull, sw, (lane & ~3) + m);
+                    } else {  // two runs: each lane computes its own
+                        const float t = __fdiv_rn(amax[m], 7.f);
+                        const __half hs = __float2half_rn(fminf(t, 65504.f));
+                        const float sv = __half2float(hs);
+                        inv_of[m] = sv > 0.f ? __frcp_rn(sv) : 0.f;
+                        sw_of[m] = __half_as_ushort(hs) | ((t >= 6.103515625e-05f && t <= 65504.f) ? 0x10000u : 0u);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < R::kRuns; ++m) {
+                const float inv = inv_of[m];
                 uint32_t z[8];
-                if (t >= 6.103515625e-05f && t <= 65504.f) {
+                if (sw_of[m] >> 16) {
                     // s is a normal half within 2^-11 of absmax / 7: |y * inv| < 7.5,
                     // so one fused multiply-add rounds the exact product, no clamp
 #pragma unroll
@@ -184,7 +219,7 @@ __global__ void __launch_bounds__(kThreads) k_kv4_encode(const uint4 *__restrict
                     }
                 }
                 word[m] = pack_nibbles(z);
-                sbits[m] = __half_as_ushort(hs);
+                sbits[m] = (uint16_t)sw_of[m];
             }
             if (row < n_rows) {
 #pragma unroll
