@@ -104,3 +104,29 @@ def test_traffic_guard_ignores_comments_only(tmp_path, monkeypatch):
     src.write_text("// header\n__global__ void k(int *p) {\n    p[0] = 2;  // store\n}\n")
     assert bench.sources_sha(("k.cu",)) != h0
 
+
+
+def test_kv_workload_bytes_and_command_line():
+    """The KV codec's line: the workload is accepted, its algorithmic bytes are
+    2 + 0.5 + 1/16 bytes per value, and the recorded traffic matches the
+    kernel's current code."""
+    w = synth.KV_WORKLOADS["kv4_128k"]
+    assert w.rows == 131072 * 4 * 2 and w.D == 128
+    assert bench.kv_bytes(w) == w.rows * w.D * 2 + w.rows * w.D // 2 + w.rows * (w.D // 32) * 2 == 343932928
+    args = bench.parse_args(["--workload", "kv4_128k", "--steps", "20", "--warmup", "5"])
+    assert args.workload == "kv4_128k"
+    for kern in ("encode", "decode"):
+        b, note = bench.measured_traffic(f"kv4_128k_{kern}")
+        assert b is not None, note
+        assert 0.5 * bench.kv_bytes(w) < b <= bench.kv_bytes(w) * 1.05
+
+
+def test_kv_reference_arm_prints_one_line(capsys):
+    args = bench.parse_args(["--impl", "reference", "--workload", "kv4_128k", "--steps", "1", "--warmup", "0",
+                             "--cpu-seconds", "0.05"])
+    bench.run_reference(args, 1, 0)
+    import json
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["workload"] == "kv4_128k"
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
